@@ -1,0 +1,216 @@
+"""Attention: the exact definition and step-by-step emulations of both modes.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+Inputs are float32 numpy arrays [B, H, N, d] (the exact upcast of the stored
+bf16/fp16 tensors).  ``heads`` selects (b, h) pairs and ``rows`` selects query
+rows, so that large workloads can be sampled; quantisation always runs over
+the full token range of every selected head, as the device does.
+
+The emulations follow the order of the method:
+
+1. quantise (``quant.quantize_head_*``);
+2. for each query row, sweep the keys in tiles of ``block_kv`` with an online
+   softmax: running max m, P~ = 2^(S - m) relative to the running max after the
+   tile, rescale factor alpha = 2^(m_old - m_new), l accumulated from the
+   unquantised P~ (FlashAttention-style streaming, which the TurboDiffusion
+   explainer, wxsanhe.com post 64219, section 1, says the method replaces);
+3. quantise P~ per tile and accumulate its product with the quantised V.
+
+Scores are carried in the base-2 domain: S2 = S * sm_scale * log2(e).
+
+Float64 is used after the codes (exact integer S for INT8, dequantised
+products, accumulations).  The FP32 rounding order of the device's two-level
+accumulator does not change these results beyond FP32 rounding, so the
+accumulation period G does not appear here.
+"""
+
+import math
+
+import numpy as np
+
+from .formats import e4m3_round, e4m3_decode, int8_quantize  # noqa: F401
+from .quant import quantize_head_i8f8, quantize_head_nvfp4, nvfp4_dequant_rows, nvfp4_quant_rows
+
+LOG2E = 1.0 / math.log(2.0)
+P_SCALE_FP8 = 448.0           # static scale of P~ in [0, 1] onto E4M3's range
+P_STAGE1_DIV = 448.0 * 6.0    # two-stage P: row max of the tile maps to 6 * 448
+
+
+def default_scale(d, sm_scale):
+    return 1.0 / math.sqrt(d) if (sm_scale is None or sm_scale <= 0) else float(sm_scale)
+
+
+def _sel(B, H, N, heads, rows):
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(H)]
+    rows = np.arange(N) if rows is None else np.asarray(rows, dtype=np.int64)
+    return heads, rows
+
+
+def _valid_mask(rows, cols, n, causal):
+    """Key j is valid for query i iff j < N and (not causal or j <= i)."""
+    m = np.broadcast_to(cols[None, :] < n, (len(rows), len(cols))).copy()
+    if causal:
+        m &= cols[None, :] <= rows[:, None]
+    return m
+
+
+def attn_exact(q, k, v, causal=False, sm_scale=None, heads=None, rows=None):
+    """O = softmax(Q K^T * sm_scale [masked]) V in float64.
+
+    Returns [len(heads), len(rows), d] float64.
+    """
+    B, H, N, d = q.shape
+    s = default_scale(d, sm_scale)
+    heads, rows = _sel(B, H, N, heads, rows)
+    out = np.empty((len(heads), len(rows), d))
+    cols = np.arange(N)
+    for t, (b, h) in enumerate(heads):
+        qh = q[b, h].astype(np.float64)[rows]
+        S = (qh @ k[b, h].astype(np.float64).T) * s
+        S = np.where(_valid_mask(rows, cols, N, causal), S, -np.inf)
+        S = S - S.max(axis=1, keepdims=True)
+        P = np.exp(S)
+        out[t] = (P @ v[b, h].astype(np.float64)) / P.sum(axis=1, keepdims=True)
+    return out
+
+
+def _online_softmax(S2, valid, tile, p_quant, pv):
+    """Generic streaming softmax over key tiles.
+
+    S2: [R, N] float64 base-2 scores; valid: [R, N] bool.
+    p_quant(P~ tile) -> (Pq tile, row factor) : quantised P and the factor that
+        multiplies the tile's contribution (1 for static scales).
+    pv(Pq, j0, j1) -> [R, d] product of the quantised P tile with V rows j0:j1.
+    Returns (acc [R, d], l [R]) with O = acc / l up to the V scale.
+    """
+    R, N = S2.shape
+    m = np.full(R, -np.inf)
+    l = np.zeros(R)
+    acc = None
+    for j0 in range(0, N, tile):
+        j1 = min(j0 + tile, N)
+        St = np.where(valid[:, j0:j1], S2[:, j0:j1], -np.inf)
+        m_new = np.maximum(m, St.max(axis=1))
+        m_use = np.where(np.isneginf(m_new), 0.0, m_new)
+        P = np.exp2(St - m_use[:, None])                 # 0 where masked
+        alpha = np.exp2(np.where(np.isneginf(m), -np.inf, m - m_use))
+        l = alpha * l + P.sum(axis=1)
+        Pq, fac = p_quant(P)
+        contrib = pv(Pq, j0, j1) * fac[:, None]
+        acc = contrib if acc is None else alpha[:, None] * acc + contrib
+        m = m_new
+    return acc, l
+
+
+def attn_online_unquantised(q, k, v, causal=False, sm_scale=None, heads=None,
+                            rows=None, block_kv=128):
+    """The same tiled online softmax with every quantiser replaced by identity.
+
+    Equal to ``attn_exact`` up to float64 rounding; pins the streaming logic.
+    """
+    B, H, N, d = q.shape
+    s = default_scale(d, sm_scale)
+    heads, rows = _sel(B, H, N, heads, rows)
+    out = np.empty((len(heads), len(rows), d))
+    cols = np.arange(N)
+    for t, (b, h) in enumerate(heads):
+        vh = v[b, h].astype(np.float64)
+        S2 = (q[b, h].astype(np.float64)[rows] @ k[b, h].astype(np.float64).T) * (s * LOG2E)
+        acc, l = _online_softmax(
+            S2, _valid_mask(rows, cols, N, causal), block_kv,
+            lambda P: (P, np.ones(P.shape[0])),
+            lambda Pq, j0, j1: Pq @ vh[j0:j1])
+        out[t] = acc / l[:, None]
+    return out
+
+
+def int8_scores(qh, kh):
+    """Exact integer S = q k^T of int8 codes (int64 accumulation)."""
+    return qh.astype(np.int64) @ kh.astype(np.int64).T
+
+
+def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
+                         block_q=128, block_kv=128):
+    """INT8 QK^T / FP8 PV emulation (the I8QK_F8PV mode).
+
+    Steps (TurboDiffusion explainer, section 1: QK in INT8, PV in FP8, outlier
+    smoothing, two-level accumulation; tag page SageAttention3 summary [17]:
+    per-block INT8 for Q/K):
+      S2[i,j] = (q8_i . k8_j) * s_q[blk(i)] * s_k[blk(j)] * sm_scale * log2 e
+      P~ tile = 2^(S2 - m_running);  p8 = E4M3(448 * P~)
+      acc     = alpha * acc + p8 @ v8;  l = alpha * l + rowsum(P~)
+      O       = acc * s_v[c] / (448 * l)
+    """
+    B, H, N, d = q.shape
+    s = default_scale(d, sm_scale)
+    heads, rows = _sel(B, H, N, heads, rows)
+    out = np.empty((len(heads), len(rows), d))
+    cols = np.arange(N)
+    for t, (b, h) in enumerate(heads):
+        z = quantize_head_i8f8(q[b, h], k[b, h], v[b, h], block_q, block_kv)
+        v8 = e4m3_decode(z["v"])
+        Sint = int8_scores(z["q"][rows], z["k"]).astype(np.float64)
+        sq_rows = z["sq"][rows // block_q].astype(np.float64)
+        sk_cols = z["sk"][cols // block_kv].astype(np.float64)
+        S2 = Sint * sq_rows[:, None] * sk_cols[None, :] * (s * LOG2E)
+        acc, l = _online_softmax(
+            S2, _valid_mask(rows, cols, N, causal), block_kv,
+            lambda P: (e4m3_round(P_SCALE_FP8 * P), np.ones(P.shape[0])),
+            lambda Pq, j0, j1: Pq @ v8[j0:j1])
+        out[t] = acc * z["sv"].astype(np.float64)[None, :] / (P_SCALE_FP8 * l[:, None])
+    return out
+
+
+def two_stage_p_nvfp4(P):
+    """Two-stage quantisation of one P~ tile [R, T] (T <= 128 keys).
+
+    Stage 1 (per row of the tile): s1 = rowmax(P~) / (448 * 6), s1 = 1 for an
+    all-zero row; P2 = P~ / s1, so the row maximum lands on 6 * 448 and the
+    second-stage E4M3 scales use their whole range.  Stage 2: NVFP4 blocks of
+    16 keys on P2.  (Tag page, SageAttention3 summary, FP4 bullets [15][16]:
+    two-stage quantisation fixes the narrow range of P's scale factors.)
+    Returns (dequantised P2 [R, T] float64, s1 [R] float64).
+    """
+    r = P.max(axis=1)
+    s1 = np.where(r > 0, r / P_STAGE1_DIV, 1.0)
+    P2 = (P / s1[:, None]).astype(np.float32)
+    T = P.shape[1]
+    codes, _, sc = nvfp4_quant_rows(P2)
+    return nvfp4_dequant_rows(codes, sc)[:, :T], s1
+
+
+def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
+                          block_kv=128):
+    """NVFP4 microscaled emulation (the NVFP4 mode).
+
+      Q^, K'^ : NVFP4 along channels;  V^ : NVFP4 along tokens
+      S2      = (Q^ K'^T) * sm_scale * log2 e          (block scales applied exactly)
+      per key tile: P~ = 2^(S2 - m_running); (P2^, s1) = two_stage_p_nvfp4(P~)
+      acc     = alpha * acc + s1 * (P2^ @ V^);  l = alpha * l + rowsum(P~)
+      O       = acc / l
+    """
+    B, H, N, d = q.shape
+    s = default_scale(d, sm_scale)
+    heads, rows = _sel(B, H, N, heads, rows)
+    out = np.empty((len(heads), len(rows), d))
+    cols = np.arange(N)
+    for t, (b, h) in enumerate(heads):
+        z = quantize_head_nvfp4(q[b, h], k[b, h], v[b, h])
+        qv = nvfp4_dequant_rows(z["q"], z["q_sc"])[:, :d]
+        kv = nvfp4_dequant_rows(z["k"], z["k_sc"])[:, :d]
+        vv = nvfp4_dequant_rows(z["vt"], z["vt_sc"])[:, :N].T      # [N, d]
+        S2 = (qv[rows] @ kv.T) * (s * LOG2E)
+        acc, l = _online_softmax(
+            S2, _valid_mask(rows, cols, N, causal), block_kv,
+            two_stage_p_nvfp4,
+            lambda Pq, j0, j1: Pq @ vv[j0:j1])
+        out[t] = acc / l[:, None]
+    return out
+
+
+def cosine(a, b):
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))

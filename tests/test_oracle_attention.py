@@ -1,0 +1,237 @@
+"""Pins for the attention oracle (no GPU): closed forms, invariants, brute force."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from oracle import quant as Qz
+from oracle.formats import e4m3_decode
+import workloads as W
+from tests import scalar_ref
+
+
+def _inputs(B, H, N, d, seed=0, dtype="bf16", causal=False, q_outlier_frac=0.0):
+    w = W.custom(B, H, N, d, dtype=dtype, causal=causal, seed=seed, q_outlier_frac=q_outlier_frac)
+    q, k, v = W.make_inputs(w)
+    return q.float().numpy(), k.float().numpy(), v.float().numpy(), w
+
+
+# --- exact attention ------------------------------------------------------------
+
+def _triple_loop(q, k, v, causal, s):
+    N, d = q.shape
+    out = np.zeros((N, d))
+    for i in range(N):
+        sc = []
+        for j in range(N):
+            if causal and j > i:
+                continue
+            sc.append((j, sum(float(q[i, c]) * float(k[j, c]) for c in range(d)) * s))
+        mx = max(x for _, x in sc)
+        den = sum(math.exp(x - mx) for _, x in sc)
+        for c in range(d):
+            out[i, c] = sum(math.exp(x - mx) * float(v[j, c]) for j, x in sc) / den
+    return out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_matches_triple_loop(causal):
+    q, k, v, _ = _inputs(1, 2, 7, 5, seed=11)
+    o = A.attn_exact(q, k, v, causal=causal, sm_scale=0.37)
+    for h in range(2):
+        ref = _triple_loop(q[0, h], k[0, h], v[0, h], causal, 0.37)
+        assert np.abs(o[h] - ref).max() < 1e-12
+
+
+def test_exact_default_scale_is_inverse_sqrt_d():
+    q, k, v, _ = _inputs(1, 1, 9, 16, seed=3)
+    a = A.attn_exact(q, k, v, sm_scale=None)
+    b = A.attn_exact(q, k, v, sm_scale=1 / 4.0)
+    assert np.array_equal(a, b)
+
+
+def test_smoothing_invariance_exact():
+    """softmax(q (k_j - mu)) == softmax(q k_j): q.mu is constant over j."""
+    q, k, v, _ = _inputs(1, 2, 200, 32, seed=5)
+    k = k.astype(np.float64)
+    mu = k.mean(axis=2, keepdims=True)
+    for causal in (False, True):
+        a = A.attn_exact(q, k, v, causal=causal)
+        b = A.attn_exact(q, k - mu, v, causal=causal)
+        assert np.abs(a - b).max() < 1e-12
+
+
+@pytest.mark.parametrize("N,causal", [(1, False), (17, True), (300, False), (300, True), (129, True)])
+def test_online_unquantised_equals_exact(N, causal):
+    q, k, v, _ = _inputs(1, 2, N, 16, seed=N)
+    a = A.attn_exact(q, k, v, causal=causal)
+    b = A.attn_online_unquantised(q, k, v, causal=causal, block_kv=128)
+    assert np.abs(a - b).max() < 1e-12
+    c = A.attn_online_unquantised(q, k, v, causal=causal, block_kv=7)
+    assert np.abs(a - c).max() < 1e-12
+
+
+def test_sampling_rows_and_heads_matches_full():
+    q, k, v, _ = _inputs(2, 3, 150, 32, seed=9)
+    full = A.attn_quant_emul_i8f8(q, k, v)
+    rows = np.array([0, 5, 127, 128, 149])
+    part = A.attn_quant_emul_i8f8(q, k, v, heads=[(1, 2), (0, 1)], rows=rows)
+    assert np.array_equal(part[0], full[5][rows])
+    assert np.array_equal(part[1], full[1][rows])
+
+
+# --- quantised emulation: closed forms ---------------------------------------------
+
+def test_i8f8_uniform_queries_give_mean_of_dequantised_v():
+    """Q = 0 -> every score 0 -> P~ = 1 -> p8 = 448 exactly -> O = mean_j(s_v * v8_j)."""
+    _, k, v, _ = _inputs(1, 1, 300, 32, seed=2)
+    q = np.zeros_like(k)
+    o = A.attn_quant_emul_i8f8(q, k, v)[0]
+    v8, sv = Qz.quant_v_fp8(v[0, 0])
+    want = (e4m3_decode(v8) * sv.astype(np.float64)[None, :]).mean(axis=0)
+    assert np.abs(o - want[None, :]).max() < 1e-12
+
+
+def test_i8f8_one_dominant_key_selects_its_row():
+    """One key with a huge score: every other P~ underflows E4M3 -> O = dequantised V of that key."""
+    N, d = 64, 16
+    rng = np.random.default_rng(0)
+    q = np.zeros((1, 1, N, d), np.float32)
+    q[..., 0] = 1.0
+    k = rng.standard_normal((1, 1, N, d)).astype(np.float32) * 0.01
+    k[0, 0, 37, 0] = 60.0
+    v = rng.standard_normal((1, 1, N, d)).astype(np.float32)
+    o = A.attn_quant_emul_i8f8(q, k, v, sm_scale=1.0)[0]
+    v8, sv = Qz.quant_v_fp8(v[0, 0])
+    want = e4m3_decode(v8[37]) * sv
+    assert np.abs(o - want[None, :]).max() < 1e-12
+
+
+def test_int8_scores_are_exact_integers():
+    rng = np.random.default_rng(4)
+    a = rng.integers(-127, 128, (9, 32)).astype(np.int8)
+    b = rng.integers(-127, 128, (11, 32)).astype(np.int8)
+    S = A.int8_scores(a, b)
+    for i in range(9):
+        for j in range(11):
+            assert S[i, j] == sum(int(a[i, c]) * int(b[j, c]) for c in range(32))
+
+
+def test_int8_block_quant_bounds():
+    q, k, v, _ = _inputs(1, 1, 300, 64, seed=6)
+    x = q[0, 0]
+    codes, s = Qz.quant_int8_blocks(x, 128)
+    assert s.shape == (3,)
+    for b in range(3):
+        blk = x[b * 128:(b + 1) * 128].astype(np.float64)
+        c = codes[b * 128:(b + 1) * 128].astype(np.float64)
+        assert np.abs(c).max() == 127
+        assert np.abs(blk - s[b] * c).max() <= s[b] * (0.5 + 127 * 2.0 ** -23)
+
+
+def test_k_mean_and_smoothing():
+    _, k, _, _ = _inputs(1, 1, 333, 32, seed=7)
+    mu = Qz.k_channel_mean(k[0, 0])
+    assert np.abs(mu.astype(np.float64) - k[0, 0].astype(np.float64).mean(axis=0)).max() <= \
+        np.abs(mu).max() * 2.0 ** -24 + 1e-30
+    kp = Qz.smooth_k(k[0, 0], mu)
+    # the K bias (std 3) is removed: the smoothed channel means are ~0
+    assert np.abs(kp.astype(np.float64).mean(axis=0)).max() < 1e-5
+    assert np.abs(k[0, 0].mean(axis=0)).max() > 0.5
+
+
+def test_v_fp8_bounds():
+    _, _, v, _ = _inputs(1, 1, 200, 32, seed=8)
+    codes, sv = Qz.quant_v_fp8(v[0, 0])
+    deq = e4m3_decode(codes) * sv.astype(np.float64)[None, :]
+    x = v[0, 0].astype(np.float64)
+    # per channel the max magnitude maps to exactly 448
+    assert np.all(np.abs(e4m3_decode(codes)).max(axis=0) == 448.0)
+    # half-ULP of E4M3: 2^-4 relative for normals, 2^-10 absolute (in code units) below
+    tol = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * sv[None, :]) * (1 + 1e-6)
+    assert np.all(np.abs(x - deq) <= tol)
+
+
+def test_nvfp4_block_bounds():
+    q, _, _, _ = _inputs(1, 1, 64, 64, seed=12)
+    x = q[0, 0]
+    codes, sc_codes, sc = Qz.nvfp4_quant_rows(x)
+    deq = Qz.nvfp4_dequant_rows(codes, sc)
+    xb = x.reshape(64, 4, 16).astype(np.float64)
+    db = deq.reshape(64, 4, 16)
+    scb = sc.astype(np.float64)[:, :, None]
+    y = np.abs(xb) / scb
+    halfgap = np.where(y < 2, 0.25, np.where(y < 4, 0.5, 1.0))
+    sat = np.maximum(0.0, np.abs(xb) - 6 * scb)
+    assert np.all(np.abs(xb - db) <= scb * halfgap + sat + 1e-12)
+    # the scale is E4M3(amax / 6): within E4M3's half-ULP of amax/6
+    amax = np.abs(xb).max(axis=2)
+    assert np.all(np.abs(sc - amax / 6) <= amax / 6 * 2.0 ** -4 + 1e-12)
+
+
+def test_two_stage_p_row_max_maps_to_6x448():
+    rng = np.random.default_rng(1)
+    P = np.exp2(-rng.uniform(0, 30, (4, 128)))
+    P[:, 5] = 2.0 ** -20           # a tile far below the running max: tiny values
+    P2, s1 = A.two_stage_p_nvfp4(P)
+    # the largest element of each row is reproduced exactly (code 6, scale 448)
+    rowmax_idx = P.argmax(axis=1)
+    for r in range(4):
+        assert P2[r, rowmax_idx[r]] * s1[r] == pytest.approx(P[r, rowmax_idx[r]], rel=1e-7)
+
+
+# --- quantised emulation vs a scalar re-statement -----------------------------------
+
+@pytest.mark.parametrize("N,d,causal,dtype", [(40, 16, False, "fp16"), (33, 32, True, "bf16")])
+def test_i8f8_matches_scalar_restatement(N, d, causal, dtype):
+    q, k, v, _ = _inputs(1, 1, N, d, seed=N, dtype=dtype, q_outlier_frac=0.05)
+    s = 1.0 / math.sqrt(d)
+    o = A.attn_quant_emul_i8f8(q, k, v, causal=causal, block_q=16, block_kv=16)[0]
+    ref = scalar_ref.i8f8_head(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, s, blk=16)
+    assert np.abs(o - np.array(ref)).max() < 1e-9
+
+
+@pytest.mark.parametrize("N,d,causal", [(40, 32, False), (37, 16, True)])
+def test_nvfp4_matches_scalar_restatement(N, d, causal):
+    q, k, v, _ = _inputs(1, 1, N, d, seed=N + 1)
+    s = 1.0 / math.sqrt(d)
+    o = A.attn_quant_emul_nvfp4(q, k, v, causal=causal, block_kv=16)[0]
+    ref = scalar_ref.nvfp4_head(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, s, blk=16)
+    assert np.abs(o - np.array(ref)).max() < 1e-9
+
+
+# --- accuracy of the schemes themselves (the criteria the GPU path is held to) -------
+
+def test_i8f8_emulation_meets_cosine_on_small_workload():
+    q, k, v = [t.float().numpy() for t in W.make_inputs(W.SMALL)]
+    e = A.attn_exact(q, k, v)
+    z = A.attn_quant_emul_i8f8(q, k, v)
+    assert A.cosine(e, z) >= 0.999
+
+
+def test_nvfp4_two_stage_p_beats_one_stage():
+    """The tag page's SageAttention3 summary ([15][16]) says the two-stage P scale
+    fixes the narrow range of P's FP8 scale factors and improves accuracy: with the
+    first stage replaced by identity the emulation must be less accurate."""
+    w = W.custom(1, 2, 1024, 128, seed=1)
+    q, k, v = [t.float().numpy() for t in W.make_inputs(w)]
+    rows = np.arange(0, 1024, 8)
+    e = A.attn_exact(q, k, v, rows=rows)
+    two = A.attn_quant_emul_nvfp4(q, k, v, rows=rows)
+    orig = A.two_stage_p_nvfp4
+
+    def one_stage(P):
+        codes, _, sc = Qz.nvfp4_quant_rows(P.astype(np.float32))
+        return Qz.nvfp4_dequant_rows(codes, sc)[:, :P.shape[1]], np.ones(P.shape[0])
+
+    try:
+        A.two_stage_p_nvfp4 = one_stage
+        one = A.attn_quant_emul_nvfp4(q, k, v, rows=rows)
+    finally:
+        A.two_stage_p_nvfp4 = orig
+    assert A.cosine(e, two) > A.cosine(e, one)
+    # measured property of the scheme on N(0,1) inputs (no outliers): about 0.982
+    assert A.cosine(e, two) > 0.975
