@@ -1,0 +1,155 @@
+"""sattn: SageAttention-style quantized attention forward for B200 (sm_100a).
+
+Python binding of the C ABI in ``include/sattn.h`` (``libsattn.so``, built
+in-tree by ``build.py``).  This module only marshals arguments: every step of
+the computation runs in the library's CUDA kernels.  It raises when the
+library is missing or a tensor is not on a CUDA device; there is no fallback.
+
+    import bit_quantized_attention_smooth_b200 as sattn
+    out = sattn.fwd(q, k, v, causal=False, mode="i8f8")     # q, k, v [B, H, N, d]
+"""
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsattn.so")
+
+MODES = {"i8f8": 0, "nvfp4": 1}
+FP16_IO = 0x100
+STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
+          3: "SATTN_ERR_WORKSPACE", 4: "SATTN_ERR_CUDA"}
+
+# Every entry point declared in include/sattn.h.
+EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
+           "sattn_status_string", "sattn_device_error", "sattn_workspace_layout")
+
+
+class SattnError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("q8", "k8", "vt8", "sq", "sk", "sv", "mu", "ksum", "vmax", "total")] + \
+               [("nv", ctypes.c_int), ("nblk", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libsattn.so (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"libsattn.so not built at {LIB_PATH}; run bit_quantized_attention_smooth_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        i, sz, vp, f = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+        L.sattn_workspace_bytes.restype = sz
+        L.sattn_workspace_bytes.argtypes = [i, i, i, i, i]
+        L.sattn_quantize.restype = i
+        L.sattn_quantize.argtypes = [vp, vp, vp, i, i, i, i, i, vp, sz, vp]
+        L.sattn_fwd_quantized.restype = i
+        L.sattn_fwd_quantized.argtypes = [vp, sz, vp, i, i, i, i, i, f, i, vp]
+        L.sattn_fwd.restype = i
+        L.sattn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+        L.sattn_status_string.restype = ctypes.c_char_p
+        L.sattn_status_string.argtypes = [i]
+        L.sattn_device_error.restype = i
+        L.sattn_device_error.argtypes = [i]
+        L.sattn_workspace_layout.restype = i
+        L.sattn_workspace_layout.argtypes = [i, i, i, i, i, ctypes.POINTER(WsLayout)]
+        _lib = L
+    return _lib
+
+
+def mode_code(mode, dtype):
+    if mode not in MODES:
+        raise ValueError(f"mode must be one of {list(MODES)}")
+    if dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("q, k, v must be bfloat16 or float16")
+    return MODES[mode] | (FP16_IO if dtype == torch.float16 else 0)
+
+
+def _check(status, what):
+    if status != 0:
+        raise SattnError(status, what)
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(q, k, v):
+    for t in (q, k, v):
+        if not t.is_cuda:
+            raise ValueError("q, k, v must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous [B, H, N, d]")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share the shape [B, H, N, d]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    return tuple(q.shape)
+
+
+def workspace_bytes(B, H, N, d, mode="i8f8", dtype=torch.bfloat16):
+    return int(lib().sattn_workspace_bytes(B, H, N, d, mode_code(mode, dtype)))
+
+
+def workspace_layout(B, H, N, d, mode="i8f8", dtype=torch.bfloat16):
+    out = WsLayout()
+    _check(lib().sattn_workspace_layout(B, H, N, d, mode_code(mode, dtype), ctypes.byref(out)),
+           "sattn_workspace_layout")
+    return {n: getattr(out, n) for n, _ in WsLayout._fields_}
+
+
+def quantize(q, k, v, mode="i8f8", workspace=None, stream=None):
+    """Quantise q, k, v into a uint8 workspace tensor (allocated when not given)."""
+    B, H, N, d = _check_qkv(q, k, v)
+    m = mode_code(mode, q.dtype)
+    nbytes = int(lib().sattn_workspace_bytes(B, H, N, d, m))
+    if nbytes == 0:
+        raise SattnError(2, "sattn_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _check(lib().sattn_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, m,
+                                workspace.data_ptr(), workspace.numel(), _stream(stream)),
+           "sattn_quantize")
+    return workspace
+
+
+def fwd_quantized(workspace, shape, causal=False, sm_scale=None, mode="i8f8", dtype=torch.bfloat16,
+                  out=None, stream=None):
+    """Attention over a workspace filled by ``quantize``; returns out [B, H, N, d]."""
+    B, H, N, d = shape
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=dtype, device=workspace.device)
+    _check(lib().sattn_fwd_quantized(workspace.data_ptr(), workspace.numel(), out.data_ptr(),
+                                     B, H, N, d, int(bool(causal)), float(sm_scale or 0.0),
+                                     mode_code(mode, dtype), _stream(stream)),
+           "sattn_fwd_quantized")
+    return out
+
+
+def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None):
+    """O = softmax(Q K^T * sm_scale) V with quantised operands (library-owned workspace)."""
+    B, H, N, d = _check_qkv(q, k, v)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
+                           int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype),
+                           _stream(stream)),
+           "sattn_fwd")
+    return out
+
+
+def device_error(clear=False):
+    """Device-side error word (0 = no bounded wait ran out); synchronises the device."""
+    return int(lib().sattn_device_error(int(bool(clear))))

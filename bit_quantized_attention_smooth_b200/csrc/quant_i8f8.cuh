@@ -1,0 +1,254 @@
+// Quantisation kernels of the INT8-QK / FP8-PV mode.
+//
+// The TurboDiffusion explainer (wxsanhe.com post 64219, section 1 "hybrid
+// attention") puts QK^T in INT8 and PV in FP8 and recovers accuracy with
+// outlier smoothing; the SageAttention tag page (reportify.cn), SageAttention3
+// summary, bullet [17], quantises Q/K per block.  Readings used here:
+//   mu[c]   = (float)( sum_n K[n,c] (exact float64 sum) / N )      per (b,h)
+//   s_q, s_k = max|x| / 127 per 128-token block (1 for an all-zero block)
+//   q8      = RNE(x / s) clamped to [-127, 127], division in IEEE float32
+//   s_v[c]  = max_n |V[n,c]| / 448 per channel (1 for an all-zero channel)
+//   v8      = E4M3_RNE_satfinite(V / s_v), written transposed [d, Nv]
+//
+// HBM-bound.  Pass 1 (kv_stats) reads K and V once and reduces per-channel
+// sums (float64 atomics: exact for bf16/fp16 inputs, so order-independent)
+// and per-channel |V| maxima.  Pass 2 reads Q, K, V once more and writes the
+// codes; every load is a coalesced 16-byte vector.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace sattn {
+
+constexpr int kBlockTokens = 128;   // quantisation block = attention tile height
+constexpr int kQuantThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ void load8(const T *p, float (&f)[8]);
+
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load8<__half>(const __half *p, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Pass 1: per-channel float64 sums of K and float32 maxima of |V|.
+// grid (ceil(N / tokens_per_cta), B*H), block 256.
+template <typename T, int D>
+__global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__restrict__ k, const T *__restrict__ v,
+                                                                 double *__restrict__ ksum,
+                                                                 unsigned *__restrict__ vmax, int N,
+                                                                 int tokens_per_cta) {
+  constexpr int LPR = D / 8;                  // threads per row (8 channels each)
+  constexpr int RPI = kQuantThreads / LPR;    // rows per iteration
+  __shared__ double s_sum[RPI][D];
+  __shared__ float s_max[RPI][D];
+
+  const int bh = blockIdx.y;
+  const int cg = threadIdx.x % LPR;
+  const int r0 = threadIdx.x / LPR;
+  const int n_begin = blockIdx.x * tokens_per_cta;
+  const int n_end = min(N, n_begin + tokens_per_cta);
+  const size_t head = static_cast<size_t>(bh) * N * D;
+
+  double acc[8];
+  float vm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    acc[i] = 0.0;
+    vm[i] = 0.f;
+  }
+  for (int n = n_begin + r0; n < n_end; n += RPI) {
+    float kf[8], vf[8];
+    load8<T>(k + head + static_cast<size_t>(n) * D + cg * 8, kf);
+    load8<T>(v + head + static_cast<size_t>(n) * D + cg * 8, vf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      acc[i] += static_cast<double>(kf[i]);
+      vm[i] = fmaxf(vm[i], fabsf(vf[i]));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    s_sum[r0][cg * 8 + i] = acc[i];
+    s_max[r0][cg * 8 + i] = vm[i];
+  }
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    double s = 0.0;
+    float m = 0.f;
+    for (int r = 0; r < RPI; ++r) {
+      s += s_sum[r][c];
+      m = fmaxf(m, s_max[r][c]);
+    }
+    atomicAdd(ksum + static_cast<size_t>(bh) * D + c, s);
+    atomicMax(vmax + static_cast<size_t>(bh) * D + c, __float_as_uint(m));  // m >= 0: bit order = value order
+  }
+}
+
+__device__ __forceinline__ float block_max_256(float v, float *s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) s_red[warp] = v;
+  __syncthreads();
+  float m = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kQuantThreads / 32; ++w) m = fmaxf(m, s_red[w]);
+  return m;
+}
+
+// Pass 2a: per-block INT8 of Q (IS_K = false) or of K - mu (IS_K = true).
+// grid (ceil(N/128), B*H), block 256.  Each thread owns a fixed group of 8
+// channels and (128 * D / 8) / 256 row positions.
+template <typename T, int D, bool IS_K>
+__global__ void __launch_bounds__(kQuantThreads) quant_qk_kernel(const T *__restrict__ x, int8_t *__restrict__ out,
+                                                                 float *__restrict__ scale,
+                                                                 const double *__restrict__ ksum,
+                                                                 float *__restrict__ mu_out, int N, int nblk) {
+  constexpr int LPR = D / 8;
+  constexpr int RPI = kQuantThreads / LPR;
+  constexpr int ITERS = kBlockTokens / RPI;
+  __shared__ float s_red[kQuantThreads / 32];
+
+  const int bh = blockIdx.y;
+  const int blk = blockIdx.x;
+  const int cg = threadIdx.x % LPR;
+  const int r0 = threadIdx.x / LPR;
+  const size_t head = static_cast<size_t>(bh) * N * D;
+
+  float mu[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mu[i] = 0.f;
+  if (IS_K) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      mu[i] = static_cast<float>(ksum[static_cast<size_t>(bh) * D + cg * 8 + i] / static_cast<double>(N));
+    if (blk == 0 && r0 == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mu_out[static_cast<size_t>(bh) * D + cg * 8 + i] = mu[i];
+    }
+  }
+
+  float val[ITERS][8];
+  float amax = 0.f;
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int n = blk * kBlockTokens + it * RPI + r0;
+    if (n < N) {
+      load8<T>(x + head + static_cast<size_t>(n) * D + cg * 8, val[it]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (IS_K) val[it][i] = __fsub_rn(val[it][i], mu[i]);
+        amax = fmaxf(amax, fabsf(val[it][i]));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) val[it][i] = 0.f;
+    }
+  }
+  amax = block_max_256(amax, s_red);
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  if (threadIdx.x == 0) scale[static_cast<size_t>(bh) * nblk + blk] = s;
+
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int n = blk * kBlockTokens + it * RPI + r0;
+    if (n < N) {
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int qi = __float2int_rn(__fdiv_rn(val[it][i], s));
+        qi = max(-127, min(127, qi));
+        w[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
+      }
+      *reinterpret_cast<uint2 *>(out + head + static_cast<size_t>(n) * D + cg * 8) = make_uint2(w[0], w[1]);
+    }
+  }
+}
+
+// Pass 2b: per-channel FP8 E4M3 of V, stored transposed vt[bh][c][token]
+// with row length Nv (N rounded up to 16).  grid (ceil(N/128), B*H), block 256.
+template <typename T, int D>
+__global__ void __launch_bounds__(kQuantThreads) quant_v_kernel(const T *__restrict__ v, uint8_t *__restrict__ vt,
+                                                                float *__restrict__ sv_out,
+                                                                const unsigned *__restrict__ vmax, int N,
+                                                                int Nv) {
+  constexpr int LPR = D / 8;
+  constexpr int RPI = kQuantThreads / LPR;
+  constexpr int ITERS = kBlockTokens / RPI;
+  constexpr int TROW = kBlockTokens + 16;  // padded smem row (bytes)
+  __shared__ __align__(16) uint8_t tile[D][TROW];
+
+  const int bh = blockIdx.y;
+  const int blk = blockIdx.x;
+  const int cg = threadIdx.x % LPR;
+  const int r0 = threadIdx.x / LPR;
+  const size_t head = static_cast<size_t>(bh) * N * D;
+
+  float sv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float m = __uint_as_float(vmax[static_cast<size_t>(bh) * D + cg * 8 + i]);
+    sv[i] = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+  }
+  if (blk == 0 && r0 == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sv_out[static_cast<size_t>(bh) * D + cg * 8 + i] = sv[i];
+  }
+
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int nl = it * RPI + r0;
+    const int n = blk * kBlockTokens + nl;
+    float f[8];
+    if (n < N) {
+      load8<T>(v + head + static_cast<size_t>(n) * D + cg * 8, f);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const uint32_t two = cvt_e4m3x2(__fdiv_rn(f[i], sv[i]), __fdiv_rn(f[i + 1], sv[i + 1]));
+      tile[cg * 8 + i][nl] = static_cast<uint8_t>(two & 0xFFu);
+      tile[cg * 8 + i + 1][nl] = static_cast<uint8_t>(two >> 8);
+    }
+  }
+  __syncthreads();
+  // D rows x 128 tokens = D * 8 chunks of 16 bytes.
+  const int tok0 = blk * kBlockTokens;
+  const int valid_chunks = min(kBlockTokens, Nv - tok0) / 16;
+  for (int idx = threadIdx.x; idx < D * 8; idx += kQuantThreads) {
+    const int c = idx >> 3;
+    const int ch = idx & 7;
+    if (ch < valid_chunks) {
+      const uint4 u = *reinterpret_cast<const uint4 *>(&tile[c][ch * 16]);
+      *reinterpret_cast<uint4 *>(vt + (static_cast<size_t>(bh) * D + c) * Nv + tok0 + ch * 16) = u;
+    }
+  }
+}
+
+}  // namespace sattn

@@ -1,0 +1,277 @@
+// C-ABI of libsattn.so: argument validation, workspace layout, TMA tensor
+// maps and kernel launches.  Declarations and contracts: include/sattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sattn.h"
+#include "attn_i8f8.cuh"
+#include "quant_i8f8.cuh"
+
+namespace sattn {
+namespace {
+
+constexpr size_t kSectionAlign = 1024;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool valid_mode(int mode) {
+  const int base = mode & ~SATTN_FP16_IO;
+  return (mode & ~(SATTN_FP16_IO | 0xFF)) == 0 && (base == SATTN_I8QK_F8PV || base == SATTN_NVFP4);
+}
+
+int check_shape(int B, int H, int N, int d, int mode) {
+  if (B < 1 || H < 1 || N < 1) return SATTN_ERR_INVALID_ARG;
+  if (!valid_mode(mode)) return SATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SATTN_ERR_UNSUPPORTED;
+  const long long total = static_cast<long long>(B) * H * N * d;
+  if (total >= (1LL << 31) || static_cast<long long>(B) * H >= 65536) return SATTN_ERR_UNSUPPORTED;
+  if ((mode & ~SATTN_FP16_IO) == SATTN_NVFP4) return SATTN_ERR_UNSUPPORTED;
+  return SATTN_OK;
+}
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sattn_ws_layout_t make_layout(int B, int H, int N, int d) {
+  sattn_ws_layout_t L;
+  std::memset(&L, 0xFF, sizeof(L));
+  const size_t BH = static_cast<size_t>(B) * H;
+  L.nblk = (N + kBlockTokens - 1) / kBlockTokens;
+  L.nv = (N + 15) / 16 * 16;
+  size_t off = 0;
+  L.q8 = off;   off = align_up(off + BH * N * d, kSectionAlign);
+  L.k8 = off;   off = align_up(off + BH * N * d, kSectionAlign);
+  L.vt8 = off;  off = align_up(off + BH * d * L.nv, kSectionAlign);
+  L.sq = off;   off = align_up(off + BH * L.nblk * sizeof(float), kSectionAlign);
+  L.sk = off;   off = align_up(off + BH * L.nblk * sizeof(float), kSectionAlign);
+  L.sv = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
+  L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
+  L.ksum = off; off += BH * d * sizeof(double);
+  L.vmax = off; off = align_up(off + BH * d * sizeof(unsigned), kSectionAlign);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D uint8 tensor [dim2][dim1][dim0] (dim0 contiguous), box {box0, box1, 1}.
+bool make_map_u8(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint64_t stride1,
+                 uint64_t stride2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {dim0, dim1, dim2};
+  const cuuint64_t strides[2] = {stride1, stride2};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D>
+int launch_quant_i8f8(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws,
+                      const sattn_ws_layout_t &L, cudaStream_t st) {
+  double *ksum = reinterpret_cast<double *>(ws + L.ksum);
+  unsigned *vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
+  if (cudaMemsetAsync(ws + L.ksum, 0, L.total - L.ksum, st) != cudaSuccess) return SATTN_ERR_CUDA;
+  const int tpc = 512;
+  kv_stats_kernel<T, D><<<dim3((N + tpc - 1) / tpc, BH), kQuantThreads, 0, st>>>(
+      static_cast<const T *>(k), static_cast<const T *>(v), ksum, vmax, N, tpc);
+  const dim3 grid(L.nblk, BH);
+  quant_qk_kernel<T, D, false><<<grid, kQuantThreads, 0, st>>>(
+      static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq),
+      nullptr, nullptr, N, L.nblk);
+  quant_qk_kernel<T, D, true><<<grid, kQuantThreads, 0, st>>>(
+      static_cast<const T *>(k), reinterpret_cast<int8_t *>(ws + L.k8), reinterpret_cast<float *>(ws + L.sk), ksum,
+      reinterpret_cast<float *>(ws + L.mu), N, L.nblk);
+  quant_v_kernel<T, D><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(v), ws + L.vt8,
+                                                        reinterpret_cast<float *>(ws + L.sv), vmax, N, L.nv);
+  return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, typename OutT>
+int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
+                     cudaStream_t st) {
+  using SL = AttnSmem<D>;
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle swqk = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map_u8(&tq, ws + L.q8, D, N, BH, D, static_cast<uint64_t>(N) * D, D, kTile, swqk) ||
+      !make_map_u8(&tk, ws + L.k8, D, N, BH, D, static_cast<uint64_t>(N) * D, D, kTile, swqk) ||
+      !make_map_u8(&tv, ws + L.vt8, N, D, BH, L.nv, static_cast<uint64_t>(L.nv) * D, kTile, D,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return SATTN_ERR_CUDA;
+  // At least ~116 KB of shared memory so that one CTA (and its 512 TMEM
+  // columns) occupies an SM.
+  const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
+  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SATTN_ERR_CUDA;
+  AttnArgs a;
+  a.sq = reinterpret_cast<const float *>(ws + L.sq);
+  a.sk = reinterpret_cast<const float *>(ws + L.sk);
+  a.sv = reinterpret_cast<const float *>(ws + L.sv);
+  a.out = out;
+  a.N = N;
+  a.nblk = L.nblk;
+  a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  kern<<<dim3(L.nblk, BH), kAttnThreads, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+}
+
+template <int D, typename OutT>
+int dispatch_attn(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, int causal, float sm,
+                  cudaStream_t st) {
+  return causal ? launch_attn_i8f8<D, true, OutT>(ws, L, out, BH, N, sm, st)
+                : launch_attn_i8f8<D, false, OutT>(ws, L, out, BH, N, sm, st);
+}
+
+// Library-owned workspace of sattn_fwd, one per device.
+struct OwnedWorkspace {
+  void *ptr = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mutex;
+OwnedWorkspace g_ws[kMaxDevices];
+
+}  // namespace
+}  // namespace sattn
+
+using namespace sattn;
+
+extern "C" {
+
+size_t sattn_workspace_bytes(int B, int H, int N, int d, int mode) {
+  if (check_shape(B, H, N, d, mode) != SATTN_OK) return 0;
+  return make_layout(B, H, N, d).total;
+}
+
+int sattn_workspace_layout(int B, int H, int N, int d, int mode, sattn_ws_layout_t *out) {
+  if (out == nullptr) return SATTN_ERR_INVALID_ARG;
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  *out = make_layout(B, H, N, d);
+  return SATTN_OK;
+}
+
+int sattn_quantize(const void *q, const void *k, const void *v, int B, int H, int N, int d, int mode,
+                   void *workspace, size_t ws_bytes, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
+  const sattn_ws_layout_t L = make_layout(B, H, N, d);
+  if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const int BH = B * H;
+  const bool fp16 = (mode & SATTN_FP16_IO) != 0;
+  if (d == 128)
+    return fp16 ? launch_quant_i8f8<__half, 128>(q, k, v, BH, N, ws, L, cs)
+                : launch_quant_i8f8<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, cs);
+  return fp16 ? launch_quant_i8f8<__half, 64>(q, k, v, BH, N, ws, L, cs)
+              : launch_quant_i8f8<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, cs);
+}
+
+int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B, int H, int N, int d, int causal,
+                        float sm_scale, int mode, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (!aligned16(out)) return SATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
+  const sattn_ws_layout_t L = make_layout(B, H, N, d);
+  if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
+  const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+  if (static_cast<const uint8_t *>(out) < ws + L.total &&
+      ws < static_cast<const uint8_t *>(out) + static_cast<size_t>(B) * H * N * d * 2)
+    return SATTN_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) sm_scale = 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const bool fp16 = (mode & SATTN_FP16_IO) != 0;
+  if (d == 128)
+    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, cs)
+                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, cs);
+  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, cs)
+              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, cs);
+}
+
+int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
+              float sm_scale, int mode, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SATTN_ERR_INVALID_ARG;
+  const size_t io_bytes = static_cast<size_t>(B) * H * N * d * 2;
+  const uint8_t *o = static_cast<const uint8_t *>(out);
+  for (const void *in : {q, k, v}) {
+    const uint8_t *p = static_cast<const uint8_t *>(in);
+    if (o < p + io_bytes && p < o + io_bytes) return SATTN_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SATTN_ERR_CUDA;
+  const size_t need = make_layout(B, H, N, d).total;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  void *ws = nullptr;
+  size_t ws_bytes = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    OwnedWorkspace &w = g_ws[dev];
+    if (w.bytes < need) {
+      if (w.ptr != nullptr && cudaFreeAsync(w.ptr, cs) != cudaSuccess) return SATTN_ERR_CUDA;
+      w.ptr = nullptr;
+      w.bytes = 0;
+      if (cudaMallocAsync(&w.ptr, need, cs) != cudaSuccess) return SATTN_ERR_CUDA;
+      w.bytes = need;
+    }
+    ws = w.ptr;
+    ws_bytes = w.bytes;
+  }
+  const int s1 = sattn_quantize(q, k, v, B, H, N, d, mode, ws, ws_bytes, stream);
+  if (s1 != SATTN_OK) return s1;
+  return sattn_fwd_quantized(ws, ws_bytes, out, B, H, N, d, causal, sm_scale, mode, stream);
+}
+
+const char *sattn_status_string(int status) {
+  switch (status) {
+    case SATTN_OK: return "SATTN_OK";
+    case SATTN_ERR_INVALID_ARG: return "SATTN_ERR_INVALID_ARG: invalid argument";
+    case SATTN_ERR_UNSUPPORTED: return "SATTN_ERR_UNSUPPORTED: unsupported shape or mode";
+    case SATTN_ERR_WORKSPACE: return "SATTN_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case SATTN_ERR_CUDA: return "SATTN_ERR_CUDA: CUDA runtime error";
+    default: return "unknown sattn status";
+  }
+}
+
+int sattn_device_error(int clear) {
+  unsigned int word = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return -1;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return -1;
+  }
+  return static_cast<int>(word);
+}
+
+}  // extern "C"

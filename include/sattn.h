@@ -1,0 +1,125 @@
+/*
+ * sattn -- SageAttention-style quantized attention forward for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libsattn.so.  All entry points are plain C: device pointers, sizes,
+ * a CUDA stream.  No entry point throws or aborts; each returns a status code
+ * (sattn_status_t) and never synchronizes the stream unless stated.
+ *
+ * The operation (TurboDiffusion explainer, wxsanhe.com post 64219, section 1
+ * "hybrid attention": QK in INT8, PV in FP8, outlier smoothing, two-level
+ * accumulation; SageAttention tag page, reportify.cn, SageAttention3 summary,
+ * bullets [15][16][17]: NVFP4 microscaling, two-stage P scale, per-block INT8):
+ *
+ *     O = softmax(Q K^T * sm_scale [+ causal mask]) V
+ *
+ * computed with quantized operands:
+ *   SATTN_I8QK_F8PV : K smoothed by its per-channel token mean; Q and K INT8
+ *                     with one float32 scale per 128-token block; V FP8 E4M3
+ *                     with one scale per channel; P FP8 E4M3 (static scale 448);
+ *                     P.V accumulated in an inner FP32 accumulator that is
+ *                     flushed into an outer FP32 accumulator every few key
+ *                     blocks (two-level accumulation).
+ *   SATTN_NVFP4     : FP4 E2M1 values with one E4M3 scale per 16 values for
+ *                     Q, K (along channels) and V (along tokens); P quantized
+ *                     in two stages (a per-row, per-key-block float32 scale,
+ *                     then NVFP4).  [not yet implemented: returns
+ *                     SATTN_ERR_UNSUPPORTED]
+ *
+ * Tensor layout (all modes): q, k, v, out are contiguous [B, H, N, d] ("BHND"),
+ * element type bf16 (default) or fp16 (mode | SATTN_FP16_IO); out has the
+ * input's element type.  Pointers must be 16-byte aligned device pointers.
+ * Supported: d in {64, 128}; N >= 1; B*H >= 1; B*H*N*d < 2^31.
+ * sm_scale <= 0 selects 1/sqrt(d).  causal masks key j > query i.
+ *
+ * Errors: invalid arguments are rejected before any launch with
+ * SATTN_ERR_INVALID_ARG / SATTN_ERR_UNSUPPORTED / SATTN_ERR_WORKSPACE.  A
+ * failed launch returns SATTN_ERR_CUDA.  Faults during execution surface at the
+ * caller's next synchronization, as with any CUDA kernel.  Every wait inside
+ * the kernels is bounded; a wait that runs out sets a device-side error word
+ * (read with sattn_device_error) and the kernel returns early with partial
+ * output.
+ */
+#ifndef SATTN_H
+#define SATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st *sattn_stream_t;
+
+typedef enum {
+  SATTN_I8QK_F8PV = 0,
+  SATTN_NVFP4 = 1,
+  SATTN_FP16_IO = 0x100 /* flag: q, k, v, out are fp16 instead of bf16 */
+} sattn_mode_t;
+
+typedef enum {
+  SATTN_OK = 0,
+  SATTN_ERR_INVALID_ARG = 1,
+  SATTN_ERR_UNSUPPORTED = 2,
+  SATTN_ERR_WORKSPACE = 3,
+  SATTN_ERR_CUDA = 4
+} sattn_status_t;
+
+/* Bytes of workspace that sattn_quantize fills for this problem and mode
+ * (0 for invalid arguments).  Depends only on (B, H, N, d, mode). */
+size_t sattn_workspace_bytes(int B, int H, int N, int d, int mode);
+
+/* Quantize q, k, v into `workspace` (device memory of at least
+ * sattn_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller).
+ * I8QK_F8PV: per-channel K mean (float64 sum of the stored values / N, rounded
+ * once to float32), per-block INT8 codes and scales of Q and of K - mean,
+ * per-channel FP8 codes and scales of V (V stored transposed, tokens
+ * contiguous).  Asynchronous on `stream`.  The workspace stays valid for any
+ * number of sattn_fwd_quantized calls with the same (B, H, N, d, mode). */
+int sattn_quantize(const void *q, const void *k, const void *v,
+                   int B, int H, int N, int d, int mode,
+                   void *workspace, size_t ws_bytes, sattn_stream_t stream);
+
+/* Fused attention over a workspace filled by sattn_quantize with the same
+ * (B, H, N, d, mode).  Writes out [B, H, N, d].  `out` must not alias the
+ * workspace.  Asynchronous on `stream`. */
+int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out,
+                        int B, int H, int N, int d, int causal, float sm_scale,
+                        int mode, sattn_stream_t stream);
+
+/* sattn_quantize followed by sattn_fwd_quantized, with a workspace that the
+ * library owns: one per device, allocated on first use with cudaMallocAsync on
+ * `stream` and grown (never shrunk) when a larger problem arrives.  Calls that
+ * share a device must be ordered (same stream, or synchronized), because they
+ * share this workspace.  `out` must not alias q, k or v. */
+int sattn_fwd(const void *q, const void *k, const void *v, void *out,
+              int B, int H, int N, int d, int causal, float sm_scale, int mode,
+              sattn_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *sattn_status_string(int status);
+
+/* Device-side error word of the current device: 0 when no kernel wait has run
+ * out of time since the last clear.  Synchronizes the device.  clear != 0
+ * resets the word to 0 after reading. */
+int sattn_device_error(int clear);
+
+/* Byte offsets of the workspace sections, for tests and tools that read the
+ * quantized operands.  Offsets not used by a mode are set to SIZE_MAX.
+ *   I8QK_F8PV: q8  int8   [B*H, N, d]        k8 int8 [B*H, N, d]
+ *              vt8 e4m3   [B*H, d, Nv]  (Nv = N rounded up to 16)
+ *              sq, sk float32 [B*H, ceil(N/128)]   sv, mu float32 [B*H, d]
+ *              ksum float64 [B*H, d], vmax uint32 [B*H, d] (scratch) */
+typedef struct {
+  size_t q8, k8, vt8, sq, sk, sv, mu, ksum, vmax, total;
+  int nv, nblk;
+} sattn_ws_layout_t;
+
+int sattn_workspace_layout(int B, int H, int N, int d, int mode, sattn_ws_layout_t *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SATTN_H */

@@ -127,8 +127,13 @@ def attn_online_unquantised(q, k, v, causal=False, sm_scale=None, heads=None,
 
 
 def int8_scores(qh, kh):
-    """Exact integer S = q k^T of int8 codes (int64 accumulation)."""
-    return qh.astype(np.int64) @ kh.astype(np.int64).T
+    """Exact integer S = q k^T of int8 codes.
+
+    Computed as a float64 matrix product: every product and partial sum is an
+    integer of magnitude <= 127 * 127 * d < 2^53, so the result is exact and
+    independent of summation order.  Returned as int64.
+    """
+    return (qh.astype(np.float64) @ kh.astype(np.float64).T).astype(np.int64)
 
 
 def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,

@@ -1,0 +1,88 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/sattn.h, and rejects bad arguments before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_quantized_attention_smooth_b200 as sattn
+from bit_quantized_attention_smooth_b200 import build as sattn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sattn.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+BF16, FP16, NVFP4 = 0, 0x100, 1
+
+
+@pytest.fixture(scope="module")
+def L():
+    sattn_build.build()
+    return sattn.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sattn_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert set(names) == set(sattn.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert L.sattn_status_string(code).startswith(b"SATTN_")
+    assert b"unknown" in L.sattn_status_string(99)
+
+
+def test_workspace_bytes_and_layout(L):
+    assert L.sattn_workspace_bytes(1, 2, 256, 64, FP16) > 0
+    assert L.sattn_workspace_bytes(1, 2, 0, 64, BF16) == 0       # N < 1
+    assert L.sattn_workspace_bytes(1, 2, 256, 96, BF16) == 0      # d unsupported
+    assert L.sattn_workspace_bytes(1, 2, 256, 64, 7) == 0         # unknown mode
+    lay = sattn.workspace_layout(1, 12, 32760, 128)
+    assert lay["nblk"] == 256 and lay["nv"] == 32768
+    bh, n, d = 12, 32760, 128
+    assert lay["k8"] - lay["q8"] >= bh * n * d
+    assert lay["sk"] - lay["sq"] >= bh * 256 * 4
+    assert lay["total"] >= lay["vmax"] + bh * d * 4
+    for key in ("q8", "k8", "vt8", "sq", "sk", "sv", "mu", "ksum"):
+        assert lay[key] % 256 == 0, key
+    assert lay["total"] == L.sattn_workspace_bytes(1, 12, 32760, 128, BF16)
+
+
+def test_invalid_arguments_rejected_before_launch(L):
+    p = ctypes.c_void_p(1 << 20)          # never dereferenced: validation fails first
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    ws = ctypes.c_void_p(1 << 21)
+    q = L.sattn_quantize
+    assert q(p, p, p, 1, 2, 256, 96, BF16, ws, 1 << 30, None) == UNSUPPORTED
+    assert q(p, p, p, 1, 2, 0, 64, BF16, ws, 1 << 30, None) == INVALID
+    assert q(p, p, p, 0, 2, 256, 64, BF16, ws, 1 << 30, None) == INVALID
+    assert q(p, p, p, 1, 2, 256, 64, 5, ws, 1 << 30, None) == INVALID
+    assert q(None, p, p, 1, 2, 256, 64, BF16, ws, 1 << 30, None) == INVALID
+    assert q(mis, p, p, 1, 2, 256, 64, BF16, ws, 1 << 30, None) == INVALID
+    assert q(p, p, p, 1, 2, 256, 64, BF16, None, 1 << 30, None) == WORKSPACE
+    assert q(p, p, p, 1, 2, 256, 64, BF16, ctypes.c_void_p((1 << 21) + 16), 1 << 30, None) == WORKSPACE
+    assert q(p, p, p, 1, 2, 256, 64, BF16, ws, 16, None) == WORKSPACE
+    assert q(p, p, p, 1, 2, 256, 64, NVFP4, ws, 1 << 30, None) == UNSUPPORTED
+    assert q(p, p, p, 1 << 16, 1, 256, 64, BF16, ws, 1 << 40, None) == UNSUPPORTED   # B*H too large
+    f = L.sattn_fwd_quantized
+    assert f(ws, 1 << 30, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
+    assert f(ws, 16, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == WORKSPACE
+    # out overlapping the workspace
+    assert f(ws, 1 << 30, ctypes.c_void_p((1 << 21) + 1024), 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
+    g = L.sattn_fwd
+    assert g(p, p, p, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
+    assert g(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
+    assert g(p, p, p, mis, 1, 2, 256, 128, 0, 0.0, 0x200, None) == INVALID   # unknown flag

@@ -5,9 +5,11 @@ holds only the input recipe (shapes, distributions, seeds) and none of the
 attention or quantisation arithmetic.
 
 Recipe (identical for every caller):
-  * ``torch.Generator('cpu').manual_seed(seed)``; draws in float32 in the order
-    q, k, k-bias, v, outlier mask, then cast to the workload dtype, so the
-    device and the oracle see the same stored tensors.
+  * one ``torch.Generator('cpu')`` per (batch, head), seeded with
+    ``seed * 1_000_003 + b * H + h``; per head it draws in float32, in order,
+    q [N, d], k [N, d], the k bias [d], v [N, d] and the outlier mask [N, d],
+    then casts to the workload dtype, so the device and the oracle see the same
+    stored tensors and any single head can be regenerated on its own.
   * Q, V ~ N(0, 1).
   * K ~ N(0, 1) + b[c], b ~ N(0, 3^2) drawn once per (batch, head) and shared
     by all tokens: the per-channel offset that K smoothing removes.
@@ -70,20 +72,46 @@ SWEEP_POINTS = [(d, n, c) for d in (64, 128) for n in (1024, 2048, 4096, 8192, 1
                 for c in (False, True)]
 
 
-def make_inputs(w: Workload, device="cpu"):
-    """Return (q, k, v) with shape [B, H, N, d] in the workload dtype."""
-    g = torch.Generator("cpu").manual_seed(w.seed)
-    shape = (w.B, w.H, w.N, w.d)
+def make_head(w: Workload, b: int, h: int):
+    """Return (q, k, v) of one (batch, head): [N, d] in the workload dtype."""
+    g = torch.Generator("cpu").manual_seed(w.seed * 1_000_003 + b * w.H + h)
+    shape = (w.N, w.d)
     q = torch.randn(shape, generator=g, dtype=torch.float32)
     k = torch.randn(shape, generator=g, dtype=torch.float32)
-    bias = torch.randn((w.B, w.H, 1, w.d), generator=g, dtype=torch.float32) * 3.0
-    k += bias
+    k += torch.randn((1, w.d), generator=g, dtype=torch.float32) * 3.0
     v = torch.randn(shape, generator=g, dtype=torch.float32)
     if w.q_outlier_frac > 0:
         mask = torch.rand(shape, generator=g, dtype=torch.float32) < w.q_outlier_frac
         q = torch.where(mask, q * w.q_outlier_mult, q)
     dt = w.torch_dtype
-    return q.to(dt).to(device), k.to(dt).to(device), v.to(dt).to(device)
+    return q.to(dt), k.to(dt), v.to(dt)
+
+
+def make_inputs(w: Workload, device="cpu"):
+    """Return (q, k, v) with shape [B, H, N, d] in the workload dtype."""
+    dt = w.torch_dtype
+    q = torch.empty((w.B, w.H, w.N, w.d), dtype=dt, device=device)
+    k = torch.empty_like(q)
+    v = torch.empty_like(q)
+    for b in range(w.B):
+        for h in range(w.H):
+            hq, hk, hv = make_head(w, b, h)
+            q[b, h].copy_(hq)
+            k[b, h].copy_(hk)
+            v[b, h].copy_(hv)
+    return q, k, v
+
+
+def make_heads_f32(w: Workload, heads):
+    """float32 numpy arrays [1, len(heads), N, d] of the selected (b, h) pairs."""
+    import numpy as np
+    qs, ks, vs = [], [], []
+    for (b, h) in heads:
+        hq, hk, hv = make_head(w, b, h)
+        qs.append(hq.float().numpy())
+        ks.append(hk.float().numpy())
+        vs.append(hv.float().numpy())
+    return (np.stack(qs)[None], np.stack(ks)[None], np.stack(vs)[None])
 
 
 def custom(B, H, N, d, dtype="bf16", causal=False, seed=0, q_outlier_frac=0.0):
