@@ -94,17 +94,25 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- oracle arm
 
-def oracle_sample(w, target_s):
+def oracle_sample(w, target_s, rows_n=None):
     """Time the CPU oracle on head 0 of the workload; rows sized to ~target_s.
 
     Returns (ops processed, seconds, rows).  Quantisation of the whole head is
     part of every sample (the oracle always quantises full heads)."""
     from oracle import attention as A
     qf, kf, vf = W.make_heads_f32(w, [(0, 0)])
+    if rows_n is not None:
+        rows = np.linspace(0, w.N - 1, rows_n).astype(np.int64)
+        t0 = time.perf_counter()
+        A.attn_quant_emul_i8f8(qf, kf, vf, rows=rows)
+        return 4.0 * rows_n * w.N * w.d, time.perf_counter() - t0, rows_n
+    A.attn_quant_emul_i8f8(qf, kf, vf, rows=np.arange(1))            # warm caches
     t0 = time.perf_counter()
-    A.attn_quant_emul_i8f8(qf, kf, vf, rows=np.arange(4))
-    t_small = time.perf_counter() - t0
-    rows_n = int(max(4, min(w.N, 4 * target_s / max(t_small, 1e-3))))
+    A.attn_quant_emul_i8f8(qf, kf, vf, rows=np.arange(65))
+    t65 = time.perf_counter() - t0
+    # linear through the origin: over-estimates the per-row cost (the time
+    # includes the head's quantisation), so the sample stays within target_s
+    rows_n = int(max(1, min(w.N, 65 * target_s / t65)))
     rows = np.linspace(0, w.N - 1, rows_n).astype(np.int64)
     t0 = time.perf_counter()
     A.attn_quant_emul_i8f8(qf, kf, vf, rows=rows)
@@ -127,12 +135,13 @@ def run_reference(args):
         return 0
     w = WORKLOAD
     per_step = min(4.0, 150.0 / max(1, args.steps + args.warmup))
+    _, _, rows_n = oracle_sample(w, per_step)            # calibration (untimed)
     for _ in range(args.warmup):
-        oracle_sample(w, per_step)
+        oracle_sample(w, per_step, rows_n)
     ops, secs = 0.0, 0.0
     rows_used = 0
     for _ in range(args.steps):
-        o, t, r = oracle_sample(w, per_step)
+        o, t, r = oracle_sample(w, per_step, rows_n)
         ops += o
         secs += t
         rows_used = r
@@ -313,7 +322,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sattn", choices=["sattn", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
