@@ -196,6 +196,15 @@ def run_gpu(args):
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    if args.profile:
+        # Profiling mode (for ncu): the same steps, no e2e leg, no CPU baseline.
+        for _ in range(args.steps):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile": True, "workload": w.name, "steps": args.steps,
+                          "device_error_word": sattn.device_error()}), flush=True)
+        return 0
 
     def barrier():
         if ws_n > 1:
@@ -324,6 +333,8 @@ def main():
     ap.add_argument("--impl", default="sattn", choices=["sattn", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run warm-up + steps of the GPU path only (for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
