@@ -24,7 +24,7 @@ STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
 
 # Every entry point declared in include/sattn.h.
 EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
-           "sattn_status_string", "sattn_device_error", "sattn_workspace_layout")
+           "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc")
 
 
 class SattnError(RuntimeError):
@@ -64,6 +64,8 @@ def lib():
         L.sattn_device_error.argtypes = [i]
         L.sattn_workspace_layout.restype = i
         L.sattn_workspace_layout.argtypes = [i, i, i, i, i, ctypes.POINTER(WsLayout)]
+        L.sattn_fwd_noalloc.restype = i
+        L.sattn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
         _lib = L
     return _lib
 

@@ -275,3 +275,57 @@ int sattn_device_error(int clear) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// sattn_fwd_noalloc: sattn_fwd for callers that cannot allocate device memory.
+//
+// Its workspace is a fixed static device array of SATTN_NOALLOC_MAX_BYTES
+// (declared below), which every GPU that loads this library holds until the
+// process exits.  Host code cannot pass the array's name to a kernel (on the
+// host it names a stand-in object, not device memory), so the first call on a
+// device, with that device current, looks the array's device address up with
+// cudaGetSymbolAddress and caches it; make that first call before any stream
+// capture.  No call allocates or frees memory.  All calls on a device share
+// the array and it keeps the last call's contents: the quantisation step
+// clears the two reduction buffers it accumulates into on every call, and
+// calls that overlap on the GPU (other streams, other host threads) race.
+namespace sattn {
+
+__device__ __align__(256) uint8_t g_noalloc_workspace[SATTN_NOALLOC_MAX_BYTES];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kMaxDevices];   // device address of the array per device, once looked up
+}  // namespace
+}  // namespace sattn
+
+extern "C" int sattn_fwd_noalloc(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
+                                 int d, int causal, float sm_scale, int mode, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SATTN_ERR_INVALID_ARG;
+  const size_t io_bytes = static_cast<size_t>(B) * H * N * d * 2;
+  const uint8_t *o = static_cast<const uint8_t *>(out);
+  for (const void *in : {q, k, v}) {
+    const uint8_t *p = static_cast<const uint8_t *>(in);
+    if (o < p + io_bytes && p < o + io_bytes) return SATTN_ERR_INVALID_ARG;
+  }
+  const size_t need = make_layout(B, H, N, d).total;
+  if (need > SATTN_NOALLOC_MAX_BYTES) return SATTN_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SATTN_ERR_CUDA;
+  void *ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_workspace) != cudaSuccess || addr == nullptr)
+        return SATTN_ERR_CUDA;
+      g_noalloc_addr[dev] = addr;
+    }
+    ws = g_noalloc_addr[dev];
+  }
+  const int s1 = sattn_quantize(q, k, v, B, H, N, d, mode, ws, SATTN_NOALLOC_MAX_BYTES, stream);
+  if (s1 != SATTN_OK) return s1;
+  return sattn_fwd_quantized(ws, SATTN_NOALLOC_MAX_BYTES, out, B, H, N, d, causal, sm_scale, mode, stream);
+}

@@ -97,6 +97,31 @@ int sattn_fwd(const void *q, const void *k, const void *v, void *out,
               int B, int H, int N, int d, int causal, float sm_scale, int mode,
               sattn_stream_t stream);
 
+/* Size of the static device workspace of sattn_fwd_noalloc: 64 MiB, enough
+ * for B*H*N*d up to about 22 million elements (e.g. B=1, H=12, N=4096, d=128). */
+#define SATTN_NOALLOC_MAX_BYTES (64ull << 20)
+
+/* sattn_fwd for callers that cannot allocate device memory.  The method has
+ * no counterpart on the pages; this is a deployment variant.  Some hosts own
+ * every byte of device memory and do not let a library allocate on its own
+ * (an inference engine that reserves its memory budget up front and loads
+ * this code as a plugin, or a process whose allocator is locked after
+ * start-up); for them this entry point takes its workspace from one static
+ * device array of SATTN_NOALLOC_MAX_BYTES that the library defines, so it
+ * never calls cudaMalloc, cudaMallocAsync, cudaFree or any allocating routine.
+ * Every GPU that loads libsattn.so holds that array until the process exits.
+ * Arguments, layout and semantics are those of sattn_fwd.  Returns
+ * SATTN_ERR_WORKSPACE, before any launch, when the problem needs more than
+ * SATTN_NOALLOC_MAX_BYTES (sattn_workspace_bytes tells).  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls
+ * on one device share the array, which keeps the previous call's contents
+ * (each call re-clears what must start at zero): calls that overlap on the GPU,
+ * from other streams or host threads, race and must be ordered by the caller. */
+int sattn_fwd_noalloc(const void *q, const void *k, const void *v, void *out,
+                      int B, int H, int N, int d, int causal, float sm_scale, int mode,
+                      sattn_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *sattn_status_string(int status);
 
