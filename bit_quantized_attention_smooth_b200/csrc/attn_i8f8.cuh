@@ -3,23 +3,33 @@
 // Method (TurboDiffusion explainer, wxsanhe.com post 64219, section 1 "hybrid
 // attention"): S = Q K^T in INT8, P V in FP8, with a two-level accumulator for
 // P V.  Per query tile of 128 rows and key tile j of 128 keys:
-//   S_int  = q8 . k8^T                       tcgen05.mma kind::i8 -> int32 TMEM
+//   S_int  = q8 . k8^T                         tcgen05.mma kind::i8 -> int32 TMEM
 //   S2     = S_int * s_q * s_k[j] * sm_scale * log2(e)
 //   m      = running row max of S2 (online softmax)
-//   P~     = 2^(S2 - m);  l += rowsum(P~)    FP32, one row per thread
-//   p8     = E4M3(448 P~)                    written to shared memory
-//   O_in  (+)= p8 . v8                       tcgen05.mma kind::f8f6f4 -> fp32 TMEM
-//   every G tiles, or before a tile that raises some row's max:
-//   O_out  = (O_out + O_in) * 2^(m_old - m_new)   (outer FP32 accumulator, TMEM)
-//   O      = O_out * s_v[c] / (448 l)
+//   P~     = 2^(S2 - m);  l = alpha l + rowsum(P~)   FP32, one row per thread
+//   p8     = E4M3(448 P~)                      -> shared memory
+//   O_in  (+)= p8 . v8                         tcgen05.mma kind::f8f6f4 -> fp32 TMEM
+// Two-level accumulation: the tensor cores accumulate O_in over a group of
+// kFlushEvery key tiles; at the start of every group the softmax threads add
+// O_in into the outer FP32 accumulator O_out (registers) and the next P V
+// overwrites O_in.  When a row's running max grows inside a group, that row's
+// O_in and O_out are rescaled by alpha = 2^(m_old - m_new) (per warp, only
+// when some lane of the warp needs it).  Both happen after P of the tile has
+// been written, when the previous P V has long completed.  Finally
+//   O = (O_out + O_in) * s_v[c] / (448 l).
 //
-// CTA = one 128-row query tile of one (b, h); 6 warps:
-//   warps 0-3  softmax / flush / epilogue (thread t owns row t = TMEM lane t)
-//   warp 4     TMA producer (Q once, then K_j and V_j through 3-stage rings)
-//   warp 5     TMEM allocator and single-thread MMA issuer
-// TMEM columns: S double buffer [0,128) [128,256), O_in [256,256+D),
-// O_out [384,384+D).  S_{j+1} = Q K_{j+1}^T runs on the tensor cores while the
-// softmax warps work on S_j; P V_j runs while they work on S_{j+1}.
+// CTA = two 128-row query tiles (A, B) of one (b, h) sharing every K/V tile;
+// 12 warps in 3 warpgroups:
+//   warps 0-3  softmax of tile A (thread t owns row t = TMEM lane t)
+//   warps 4-7  softmax of tile B (same lanes, other TMEM columns)
+//   warp 8     TMA producer (Q tiles once, then K_j and V_j through 3-stage rings)
+//   warp 9     TMEM allocator and single-thread MMA issuer
+//   warps 10-11 idle (they complete warpgroup 2, which gives its registers to
+//              the softmax warpgroups through setmaxnreg)
+// Two softmax warps per SM sub-partition hide each other's latency.  TMEM
+// columns: S_A [0,128), S_B [128,256), O_in_A [256,256+D), O_in_B
+// [256+D, 256+2D).  Each softmax warp reads its S twice (row max, then P), so
+// that the 128 outer-accumulator registers and one 32-column chunk fit.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -30,9 +40,15 @@
 namespace sattn {
 
 constexpr int kTile = 128;          // query rows and keys per tile
+constexpr int kQTiles = 2;          // query tiles per CTA
 constexpr int kKVStages = 3;
 constexpr int kFlushEvery = 4;      // G: key tiles per inner accumulation group
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 384;       // 3 warpgroups
+constexpr int kSoftmaxRegs = 216;       // per thread, softmax warpgroups 0 and 1
+constexpr int kControlRegs = 64;        // per thread, warpgroup 2 (TMA, MMA, 2 idle warps)
+// setmaxnreg moves registers between warpgroups of the block; the split must
+// fit in what the block was launched with (threads x launch registers).
+constexpr int kRegsNeeded = 256 * kSoftmaxRegs + 128 * kControlRegs;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
 
 struct AttnArgs {
@@ -51,16 +67,16 @@ struct AttnSmem {
   static constexpr int kKBytes = kTile * D;
   static constexpr int kVBytes = D * kTile;
   static constexpr int kPBytes = kTile * kTile;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQBytes;
-  static constexpr int kV = kK + kKVStages * kKBytes;
-  static constexpr int kP = kV + kKVStages * kVBytes;
-  static constexpr int kBar = kP + 2 * kPBytes;
-  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2],
-  // s_free[2], p_full[2], p_free[2], vote, drain
-  static constexpr int kNumBars = 1 + 4 * kKVStages + 8 + 2;
+  static constexpr int kQ = 0;                                   // [2] query tiles
+  static constexpr int kK = kQ + kQTiles * kQBytes;              // [stages]
+  static constexpr int kV = kK + kKVStages * kKBytes;            // [stages]
+  static constexpr int kP = kV + kKVStages * kVBytes;            // [2 tiles][2 buffers]
+  static constexpr int kBar = kP + kQTiles * 2 * kPBytes;
+  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
+  // p_full[2][2], pv_done[2][2], drain
+  static constexpr int kNumBars = 1 + 4 * kKVStages + 2 + 2 + 4 + 4 + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kBytes = kMisc + 64;
+  static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
 };
 
@@ -77,47 +93,48 @@ __device__ __forceinline__ uint32_t pack2_out<__half>(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Bounded wait used only while draining in-flight copies on an abort path.
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
-  const unsigned long long t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_error_word, kErrWaitTimeout);
-      return;
-    }
+// Sentinel for a masked score; |q8 . k8| <= 127 * 127 * 128 < 2^22, so no
+// real INT8 score takes this value.
+constexpr uint32_t kMaskedScore = 0x80000000u;
+// int32 -> float without a conversion instruction: for |s| < 2^22 the float
+// with bits (s + 0x4B400000) equals 12582912 + s exactly.
+constexpr int kMagicI = 0x4B400000;
+constexpr float kMagicF = 12582912.0f;
+
+__device__ __forceinline__ void mask_chunk(uint32_t (&s)[32], int kv0, int N, bool causal, int row_g) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int kv = kv0 + i;
+    if (kv >= N || (causal && kv > row_g)) s[i] = kMaskedScore;
   }
 }
 
-// Sentinel for a masked score; |q8 . k8| <= 127 * 127 * 128 < 2^21, so no
-// real INT8 score takes this value.
-constexpr uint32_t kMaskedScore = 0x80000000u;
-
-// One row of 448 * P~ = 2^(S2 - m + log2 448) -> E4M3 codes into the row's
-// 128-byte line of the P tile, in the 128-byte-swizzled K-major layout the
-// MMA reads (16-byte chunk c of row r stored at chunk c ^ (r mod 8)).
-// Accumulates the unquantised values into l448.
+// 32 scores -> 32 E4M3 codes of 448 P~ (two 16-byte chunks of the row's
+// 128-byte line in the 128-byte-swizzled K-major layout the MMA reads:
+// 16-byte chunk c of row r lives at chunk c ^ (r mod 8)); returns the sum of
+// the unquantised 448 P~.
 template <bool MASKED>
-__device__ __forceinline__ void write_p_row(const uint32_t (&S)[4][32], float c, float moff, uint8_t *prow, int r,
-                                            float &l448) {
+__device__ __forceinline__ float p_chunk(const uint32_t (&s)[32], float c, float moff, uint8_t *prow, int c16,
+                                         int r) {
+  float sum = 0.f;
+  uint32_t w[8];
 #pragma unroll
-  for (int c16 = 0; c16 < 8; ++c16) {
-    uint32_t w4[4];
+  for (int q = 0; q < 8; ++q) {
+    float p[4];
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      float p[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int idx = c16 * 16 + q4 * 4 + e;
-        const uint32_t sv = S[idx >> 5][idx & 31];
-        float x = fmaf(static_cast<float>(static_cast<int>(sv)), c, -moff);
-        if (MASKED) x = (sv == kMaskedScore) ? -INFINITY : x;
-        p[e] = ex2_approx(x);
-        l448 += p[e];
-      }
-      w4[q4] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t sv = s[q * 4 + e];
+      const float sf = __int_as_float(static_cast<int>(sv) + kMagicI) - kMagicF;   // exact
+      float x = fmaf(sf, c, -moff);
+      if (MASKED) x = (sv == kMaskedScore) ? -INFINITY : x;
+      p[e] = ex2_approx(x);
     }
-    *reinterpret_cast<uint4 *>(prow + ((c16 ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    sum += (p[0] + p[1]) + (p[2] + p[3]);
+    w[q] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
   }
+  *reinterpret_cast<uint4 *>(prow + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4 *>(prow + (((c16 + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+  return sum;
 }
 
 template <int D, bool CAUSAL, typename OutT>
@@ -126,28 +143,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
   using L = AttnSmem<D>;
   static_assert(D == 64 || D == 128, "head dim");
-  constexpr int S_COL0 = 0, S_COL1 = 128, O_IN = 256, O_OUT = 384;
   constexpr uint32_t kTmemCols = 512;
+  constexpr int kOin0 = 256;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem + L::kQ;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
   uint64_t *q_full = bars;
   uint64_t *k_full = bars + 1;
   uint64_t *k_empty = k_full + kKVStages;
   uint64_t *v_full = k_empty + kKVStages;
   uint64_t *v_empty = v_full + kKVStages;
-  uint64_t *s_full = v_empty + kKVStages;
-  uint64_t *s_free = s_full + 2;
-  uint64_t *p_full = s_free + 2;
-  uint64_t *p_free = p_full + 2;
-  uint64_t *vote_bar = p_free + 2;
-  uint64_t *drain_bar = vote_bar + 1;
+  uint64_t *s_full = v_empty + kKVStages;   // [tile]
+  uint64_t *s_free = s_full + 2;            // [tile]
+  uint64_t *p_full = s_free + 2;            // [tile * 2 + buffer]
+  uint64_t *pv_done = p_full + 4;           // [tile * 2 + buffer]
+  uint64_t *drain_bar = pv_done + 4;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
-  volatile int *pv_acc = reinterpret_cast<volatile int *>(smem + L::kMisc + 8);     // [2]
-  volatile int *votes = reinterpret_cast<volatile int *>(smem + L::kMisc + 16);     // [2][4]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -155,16 +168,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int bh = blockIdx.y;
   const int N = args.N;
   const int nkv_all = args.nblk;
-  const int qt = CAUSAL ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
-                        : static_cast<int>(blockIdx.x);
-  const int nkv = CAUSAL ? min(qt + 1, nkv_all) : nkv_all;
+  const int pair = CAUSAL ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
+                          : static_cast<int>(blockIdx.x);
+  int qt_of[kQTiles], nkv_of[kQTiles];
+#pragma unroll
+  for (int x = 0; x < kQTiles; ++x) {
+    qt_of[x] = pair * kQTiles + x;
+    nkv_of[x] = qt_of[x] >= nkv_all ? 0 : (CAUSAL ? min(qt_of[x] + 1, nkv_all) : nkv_all);
+  }
+  const int nkv_max = max(nkv_of[0], nkv_of[1]);
 
   // ------------------------------------------------------------ set-up
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (tid == 128) {
+  if (tid == 256) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(&k_full[s], 1);
@@ -172,18 +191,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);   // one arrival per softmax warp
-      mbar_init(&p_full[b], 4);
-      mbar_init(&p_free[b], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&s_free[x], 4);   // one arrival per softmax warp of the tile
     }
-    mbar_init(vote_bar, 4);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (tid == 160) {
+  if (tid == 288) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -193,21 +213,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp >= 8) {
+    regs_decrease<kControlRegs>();
+    if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       int last_j = -1;
-      mbar_arrive_expect_tx(q_full, L::kQBytes);
-      tma_load_3d(sQ, &tm_q, q_full, 0, qt * kTile, bh);
-      for (int j = 0; j < nkv; ++j) {
+      const int nq = nkv_of[1] > 0 ? 2 : 1;             // tile B may lie past the last token
+      mbar_arrive_expect_tx(q_full, nq * L::kQBytes);
+      for (int x = 0; x < nq; ++x)
+        tma_load_3d(smem + L::kQ + x * L::kQBytes, &tm_q, q_full, 0, qt_of[x] * kTile, bh);
+      for (int j = 0; j < nkv_max; ++j) {
         const int s = j % kKVStages;
         const uint32_t ph = (j / kKVStages) & 1;
         if (!mbar_wait(&k_empty[s], ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[s], L::kKBytes);
         tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
         if (!mbar_wait(&v_empty[s], ph ^ 1, abort_flag)) {
-          // K_j is in flight without its V_j: drain it before leaving.
-          drain_wait(&k_full[s], ph);
+          drain_wait(&k_full[s], ph);   // K_j is in flight without its V_j
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kVBytes);
@@ -225,48 +248,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+    } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescQK = idesc_i8_s32(kTile, kTile);
       constexpr uint32_t kIdescPV = idesc_e4m3_f32(kTile, D);
-      const uint32_t sQ_addr = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int s = j % kKVStages;
-          const int b = j & 1;
-          ok = mbar_wait(&k_full[s], (j / kKVStages) & 1, abort_flag) &&
-               mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t sK_addr = smem_u32(smem + L::kK + s * L::kKBytes);
-          const uint32_t d_tmem = tmem + (b ? S_COL1 : S_COL0);
+      for (int j = 0; ok && j <= nkv_max; ++j) {
+        bool k_ready = false, v_ready = false;
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8(d_tmem, sdesc_kmajor<D>(sQ_addr + kk * 32), sdesc_kmajor<D>(sK_addr + kk * 32), kIdescQK,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(&s_full[b]);
-          mma_commit(&k_empty[s]);
-        }
-        if (j > 0) {
-          const int t = j - 1;
-          const int s = t % kKVStages;
-          const int b = t & 1;
-          ok = mbar_wait(&v_full[s], (t / kKVStages) & 1, abort_flag) &&
-               mbar_wait(&p_full[b], (t >> 1) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t acc = static_cast<uint32_t>(pv_acc[b]);
-          const uint32_t sP_addr = smem_u32(smem + L::kP + b * L::kPBytes);
-          const uint32_t sV_addr = smem_u32(smem + L::kV + s * L::kVBytes);
+        for (int x = 0; x < kQTiles && ok; ++x) {
+          if (j < nkv_of[x]) {                              // S_x = Q_x K_j^T
+            const int s = j % kKVStages;
+            if (!k_ready) {
+              ok = mbar_wait(&k_full[s], (j / kKVStages) & 1, abort_flag);
+              k_ready = true;
+            }
+            ok = ok && mbar_wait(&s_free[x], (j & 1) ^ 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t sQ = smem_u32(smem + L::kQ + x * L::kQBytes);
+            const uint32_t sK = smem_u32(smem + L::kK + s * L::kKBytes);
 #pragma unroll
-          for (int kk = 0; kk < kTile / 32; ++kk)
-            mma_f8f6f4(tmem + O_IN, sdesc_kmajor<128>(sP_addr + kk * 32), sdesc_kmajor<128>(sV_addr + kk * 32),
-                       kIdescPV, (acc | (kk > 0 ? 1u : 0u)));
-          mma_commit(&p_free[b]);
-          mma_commit(&v_empty[s]);
+            for (int kk = 0; kk < D / 32; ++kk)
+              mma_i8(tmem + x * kTile, sdesc_kmajor<D>(sQ + kk * 32), sdesc_kmajor<D>(sK + kk * 32), kIdescQK,
+                     kk > 0 ? 1u : 0u);
+            mma_commit(&s_full[x]);
+          }
+          if (j >= 1 && j - 1 < nkv_of[x]) {                // O_in_x (+)= P_x(j-1) V_{j-1}
+            const int t = j - 1;
+            const int s = t % kKVStages;
+            const int pb = x * 2 + (t & 1);
+            if (!v_ready) {
+              ok = mbar_wait(&v_full[s], (t / kKVStages) & 1, abort_flag);
+              v_ready = true;
+            }
+            ok = ok && mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t acc = (t % kFlushEvery) != 0 ? 1u : 0u;
+            const uint32_t sP = smem_u32(smem + L::kP + pb * L::kPBytes);
+            const uint32_t sV = smem_u32(smem + L::kV + s * L::kVBytes);
+#pragma unroll
+            for (int kk = 0; kk < kTile / 32; ++kk)
+              mma_f8f6f4(tmem + kOin0 + x * D, sdesc_kmajor<128>(sP + kk * 32), sdesc_kmajor<128>(sV + kk * 32),
+                         kIdescPV, acc | (kk > 0 ? 1u : 0u));
+            mma_commit(&pv_done[pb]);
+          }
         }
+        if (!ok) break;
+        if (k_ready) mma_commit(&k_empty[j % kKVStages]);
+        if (v_ready) mma_commit(&v_empty[(j - 1) % kKVStages]);
       }
       if (!ok) {
         // Let every MMA issued so far finish before TMEM is released.
@@ -275,136 +307,127 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     __syncwarp();
+    }
   } else {
+    regs_increase<kSoftmaxRegs>();
     // ---------------------------------------------------------- softmax warps
-    const int r = tid;                                  // row in tile == TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int x = warp >> 2;                            // query tile of this warp
+    const int wq = warp & 3;                            // TMEM lane quarter
+    const int r = wq * 32 + lane;                       // row in tile == TMEM lane
+    const int qt = qt_of[x];
+    const int nkv = nkv_of[x];
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_base + x * kTile;
+    const uint32_t o_tmem = tmem + lane_base + kOin0 + x * D;
     const int row_g = qt * kTile + r;
-    const float cq = args.sq[static_cast<size_t>(bh) * args.nblk + qt] * args.sm_log2;
+    const float cq = nkv > 0 ? args.sq[static_cast<size_t>(bh) * args.nblk + qt] * args.sm_log2 : 0.f;
     const float *sk = args.sk + static_cast<size_t>(bh) * args.nblk;
+    uint8_t *p_base = smem + L::kP + (x * 2) * L::kPBytes + r * 128;
+
+    float o_out[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) o_out[i] = 0.f;
     float m_ref = -INFINITY;
     float l448 = 0.f;          // sum of 448 * P~ (the static FP8 scale folded in)
-    int glen = 0;              // key tiles in the current inner group
-    bool have_out = false;
     bool ok = true;
 
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+    for (int j = 0; j < nkv; ++j) {
+      if (!mbar_wait(&s_full[x], j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t S[4][32];
-      const uint32_t s_tmem = tmem + lane_base + (b ? S_COL1 : S_COL0);
+      const bool masked = ((j == nkv_all - 1) && (N & (kTile - 1))) || (CAUSAL && j == qt);
+
+      // pass 1: row max of the integer scores (a rolled loop over 32-column
+      // chunks keeps the loop body small enough for the instruction cache)
+      int smax = INT_MIN;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t s[32];
+        tmem_ld_32x32b_x32(s_tmem + ch * 32, s);
+        tmem_ld_wait(s);
+        if (masked) mask_chunk(s, j * kTile + ch * 32, N, CAUSAL, row_g);
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld_32x32b_x32(s_tmem + ch * 32, S[ch]);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(S[ch]);
+        for (int i = 0; i < 32; i += 2) smax = max(smax, max(static_cast<int>(s[i]), static_cast<int>(s[i + 1])));
+      }
+      const float c = cq * sk[j];
+      const float m_new = fmaxf(m_ref, static_cast<float>(smax) * c);
+      const float alpha = ex2_approx(m_ref - m_new);    // 0 at the first tile (m_ref = -inf)
+      const float moff = m_new - kLog2_448;
+
+      // pass 2: P~ -> E4M3 into P buffer (j & 1), once P V of tile j-2 has read it
+      const int pb = x * 2 + (j & 1);
+      if (!mbar_wait(&pv_done[pb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      uint8_t *prow = p_base + (j & 1) * L::kPBytes;
+      float tsum = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t s[32];
+        tmem_ld_32x32b_x32(s_tmem + ch * 32, s);
+        tmem_ld_wait(s);
+        if (masked) {
+          mask_chunk(s, j * kTile + ch * 32, N, CAUSAL, row_g);
+          tsum += p_chunk<true>(s, c, moff, prow, ch * 2, r);
+        } else {
+          tsum += p_chunk<false>(s, c, moff, prow, ch * 2, r);
+        }
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
+      if (lane == 0) mbar_arrive(&s_free[x]);            // S_x may be overwritten by Q_x K_{j+1}^T
+      l448 = fmaf(alpha, l448, tsum);
 
-      // Mask keys beyond N and, for causal, keys after the query.
-      const bool tail_tile = (j == nkv_all - 1) && (N & (kTile - 1));
-      const bool masked_tile = tail_tile || (CAUSAL && j == qt);
-      if (masked_tile) {
+      // two-level accumulation: flush O_in at a group start, or rescale on a max increase
+      const bool boundary = j > 0 && (j % kFlushEvery) == 0;
+      const bool grow = __any_sync(0xffffffffu, j > 0 && m_new > m_ref);
+      if (boundary || grow) {
+        const int t = j - 1;
+        if (!mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
+          tmem_ld_wait(o);
+          if (boundary) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int kv = j * kTile + ch * 32 + i;
-            if (kv >= N || (CAUSAL && kv > row_g)) S[ch][i] = kMaskedScore;
-          }
-      }
-      int smax = INT_MIN;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) smax = max(smax, static_cast<int>(S[ch][i]));
-      const float c = cq * sk[j];
-      const float mt = static_cast<float>(smax) * c;
-
-      // CTA-wide vote: does any row's max grow?  Votes go through shared
-      // memory and a bounded mbarrier round (no unbounded bar.sync).
-      const bool grow = __any_sync(0xffffffffu, mt > m_ref);
-      if (lane == 0) votes[(j & 1) * 4 + warp] = grow ? 1 : 0;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(vote_bar);
-      if (!mbar_wait(vote_bar, j & 1, abort_flag)) { ok = false; break; }
-      const bool any_grow = (votes[(j & 1) * 4 + 0] | votes[(j & 1) * 4 + 1] | votes[(j & 1) * 4 + 2] |
-                             votes[(j & 1) * 4 + 3]) != 0;
-
-      if (any_grow || glen == kFlushEvery) {
-        const float m_new = fmaxf(m_ref, mt);
-        const float alpha = ex2_approx(m_ref - m_new);   // 0 when m_ref = -inf
-        if (glen > 0) {
-          // The group's last P V (tile j-1) must be complete before O_in is read.
-          const int t = j - 1;
-          if (!mbar_wait(&p_free[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t oi[32], oo[32];
-            tmem_ld_32x32b_x32(tmem + lane_base + O_IN + ch * 32, oi);
-            if (have_out) {
-              tmem_ld_32x32b_x32(tmem + lane_base + O_OUT + ch * 32, oo);
-              tmem_ld_wait(oo);
-            }
-            tmem_ld_wait(oi);
+            for (int i = 0; i < 32; ++i)
+              o_out[ch * 32 + i] = alpha * (o_out[ch * 32 + i] + __uint_as_float(o[i]));
+          } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float prev = have_out ? __uint_as_float(oo[i]) : 0.f;
-              oo[i] = __float_as_uint((prev + __uint_as_float(oi[i])) * alpha);
+              o_out[ch * 32 + i] *= alpha;
+              o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             }
-            tmem_st_32x32b_x32(tmem + lane_base + O_OUT + ch * 32, oo);
+            tmem_st_32x32b_x32(o_tmem + ch * 32, o);
           }
-          tmem_st_wait();
-          have_out = true;
         }
-        l448 *= alpha;
-        m_ref = m_new;
-        glen = 0;
+        if (!boundary) tmem_st_wait();
       }
-
-      // P~ * 448 = 2^(S2 - m + log2 448), quantised to E4M3 into P buffer b
-      // (after P V of tile j-2 has finished reading it).
-      if (!mbar_wait(&p_free[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      const float moff = m_ref - kLog2_448;
-      uint8_t *prow = smem + L::kP + b * L::kPBytes + r * 128;
-      if (masked_tile)
-        write_p_row<true>(S, c, moff, prow, r, l448);
-      else
-        write_p_row<false>(S, c, moff, prow, r, l448);
-      fence_proxy_async_smem();
+      fence_proxy_async_smem();                          // P writes -> async proxy (MMA)
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        if (warp == 0) pv_acc[b] = glen > 0 ? 1 : 0;
-        mbar_arrive(&p_full[b]);
-      }
-      ++glen;
+      if (lane == 0) mbar_arrive(&p_full[pb]);
+      m_ref = m_new;
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok) {
+    if (ok && nkv > 0) {
       const int t = nkv - 1;
-      if (mbar_wait(&p_free[t & 1], (t >> 1) & 1, abort_flag)) {
+      if (mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) {
         tc_fence_after();
         const float inv_l = 1.f / l448;
         const float *sv = args.sv + static_cast<size_t>(bh) * D;
         OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D;
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t oi[32], oo[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + O_IN + ch * 32, oi);
-          if (have_out) {
-            tmem_ld_32x32b_x32(tmem + lane_base + O_OUT + ch * 32, oo);
-            tmem_ld_wait(oo);
-          }
-          tmem_ld_wait(oi);
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
+          tmem_ld_wait(o);
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float o0 = (have_out ? __uint_as_float(oo[i]) : 0.f) + __uint_as_float(oi[i]);
-            const float o1 = (have_out ? __uint_as_float(oo[i + 1]) : 0.f) + __uint_as_float(oi[i + 1]);
-            packed[i >> 1] = pack2_out<OutT>(o0 * sv[ch * 32 + i] * inv_l, o1 * sv[ch * 32 + i + 1] * inv_l);
+            const float o0 = (o_out[ch * 32 + i] + __uint_as_float(o[i])) * sv[ch * 32 + i] * inv_l;
+            const float o1 = (o_out[ch * 32 + i + 1] + __uint_as_float(o[i + 1])) * sv[ch * 32 + i + 1] * inv_l;
+            packed[i >> 1] = pack2_out<OutT>(o0, o1);
           }
           if (row_g < N) {
             uint4 *dst = reinterpret_cast<uint4 *>(orow + ch * 32);
@@ -420,7 +443,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -13,18 +13,14 @@ namespace sattn {
 __device__ unsigned int g_error_word;
 constexpr unsigned kErrWaitTimeout = 1u;
 
-// Wall-clock bound of one wait (nanoseconds of %globaltimer).  No wait in
-// these kernels legitimately lasts more than microseconds.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Bound of one wait, in SM clock cycles (about 2-4 s at 1-2 GHz).  No wait in
+// these kernels legitimately lasts more than microseconds.  The cycle counter
+// is cheap to read; it is read only every kWaitCheckEvery spins.
+constexpr long long kWaitLimitCycles = 4000000000ll;
+constexpr uint32_t kWaitCheckEvery = 256;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_timer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 // ---------------------------------------------------------------- mbarrier
@@ -54,20 +50,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits until the phase with parity `parity` of `bar` has completed.  Gives up
-// after kWaitLimitNs or when `abort_flag` (CTA shared) becomes non-zero;
+// after kWaitLimitCycles or when `abort_flag` (CTA shared) becomes non-zero;
 // on time-out it records kErrWaitTimeout in g_error_word and raises the abort
 // flag so that every role of the CTA leaves its loop.  Returns false when it
 // gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_timer_ns();
-  while (true) {
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if ((i % kWaitCheckEvery) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitLimitCycles) {
+        atomicOr(&g_error_word, kErrWaitTimeout);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used only to drain work already
+// in flight (copies, MMAs) before a CTA that gave up releases its resources.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  const long long t0 = clock64();
+  for (uint32_t i = 1; !mbar_try_wait(bar, parity); ++i) {
+    if ((i % kWaitCheckEvery) == 0 && clock64() - t0 > kWaitLimitCycles) {
       atomicOr(&g_error_word, kErrWaitTimeout);
-      *abort_flag = 1;
-      return false;
+      return;
     }
   }
 }
@@ -97,6 +107,19 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
       : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
+}
+
+// ---------------------------------------------------------------- register split
+// Warpgroup-wide change of the registers each thread owns.  An increase takes
+// registers that other warpgroups of the block released with a decrease; the
+// host checks before launch that the block's launch registers cover the split.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------- TMA

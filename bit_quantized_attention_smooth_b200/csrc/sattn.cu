@@ -122,12 +122,17 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
       !make_map_u8(&tv, ws + L.vt8, N, D, BH, L.nv, static_cast<uint64_t>(L.nv) * D, kTile, D,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return SATTN_ERR_CUDA;
-  // At least ~116 KB of shared memory so that one CTA (and its 512 TMEM
-  // columns) occupies an SM.
+  // More than half of the SM's shared memory: one CTA (and its 512 TMEM
+  // columns) per SM.
   const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
   auto kern = attn_i8f8_kernel<D, CAUSAL, OutT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SATTN_ERR_CUDA;
+  // The kernel's setmaxnreg split must fit in its launch registers, or its
+  // register increase would never be granted.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return SATTN_ERR_CUDA;
+  if (static_cast<long long>(fa.numRegs) * kAttnThreads < kRegsNeeded) return SATTN_ERR_CUDA;
   AttnArgs a;
   a.sq = reinterpret_cast<const float *>(ws + L.sq);
   a.sk = reinterpret_cast<const float *>(ws + L.sk);
@@ -136,7 +141,7 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
   a.N = N;
   a.nblk = L.nblk;
   a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
-  kern<<<dim3(L.nblk, BH), kAttnThreads, smem, st>>>(tq, tk, tv, a);
+  kern<<<dim3((L.nblk + kQTiles - 1) / kQTiles, BH), kAttnThreads, smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
