@@ -97,7 +97,10 @@ __device__ __forceinline__ uint32_t pack2_out<__half>(float a, float b) {
 // real INT8 score takes this value.
 constexpr uint32_t kMaskedScore = 0x80000000u;
 // int32 -> float without a conversion instruction: for |s| < 2^22 the float
-// with bits (s + 0x4B400000) equals 12582912 + s exactly.
+// with bits (s + 0x4B400000) equals 12582912 + s exactly.  The exponent
+// argument 2^(s c - m') is then one FMA: (12582912 + s) c - (12582912 c + m').
+// Rounding the constant costs at most c/2 in the exponent, i.e. half of one
+// integer score step, far below the INT8 quantisation error of the scores.
 constexpr int kMagicI = 0x4B400000;
 constexpr float kMagicF = 12582912.0f;
 
@@ -109,32 +112,51 @@ __device__ __forceinline__ void mask_chunk(uint32_t (&s)[32], int kv0, int N, bo
   }
 }
 
+// Maximum of 32 signed integer scores as a balanced tree (depth 5), so that
+// the comparisons of one chunk are independent instead of one serial chain.
+__device__ __forceinline__ int tree_max32(const uint32_t (&s)[32]) {
+  int m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m[i] = max(static_cast<int>(s[i]), static_cast<int>(s[i + 16]));
+#pragma unroll
+  for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = max(m[i], m[i + w]);
+  return m[0];
+}
+
 // 32 scores -> 32 E4M3 codes of 448 P~ (two 16-byte chunks of the row's
 // 128-byte line in the 128-byte-swizzled K-major layout the MMA reads:
-// 16-byte chunk c of row r lives at chunk c ^ (r mod 8)); returns the sum of
-// the unquantised 448 P~.
+// 16-byte chunk c of row r lives at chunk c ^ (r mod 8)); accumulates the
+// unquantised 448 P~ into sum2 (two partial sums).
+// b = 12582912 c + (m - log2 448).
 template <bool MASKED>
-__device__ __forceinline__ float p_chunk(const uint32_t (&s)[32], float c, float moff, uint8_t *prow, int c16,
-                                         int r) {
-  float sum = 0.f;
+__device__ __forceinline__ void p_chunk(const uint32_t (&s)[32], float c, float b, uint8_t *prow, int c16, int r,
+                                        float2 &sum2) {
+  const float2 c2 = make_float2(c, c);
+  const float2 nb2 = make_float2(-b, -b);
   uint32_t w[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    float p[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t sv = s[q * 4 + e];
-      const float sf = __int_as_float(static_cast<int>(sv) + kMagicI) - kMagicF;   // exact
-      float x = fmaf(sf, c, -moff);
-      if (MASKED) x = (sv == kMaskedScore) ? -INFINITY : x;
-      p[e] = ex2_approx(x);
+    float2 x01 = ffma2(make_float2(__int_as_float(static_cast<int>(s[4 * q]) + kMagicI),
+                                   __int_as_float(static_cast<int>(s[4 * q + 1]) + kMagicI)),
+                       c2, nb2);
+    float2 x23 = ffma2(make_float2(__int_as_float(static_cast<int>(s[4 * q + 2]) + kMagicI),
+                                   __int_as_float(static_cast<int>(s[4 * q + 3]) + kMagicI)),
+                       c2, nb2);
+    if (MASKED) {
+      if (s[4 * q] == kMaskedScore) x01.x = -INFINITY;
+      if (s[4 * q + 1] == kMaskedScore) x01.y = -INFINITY;
+      if (s[4 * q + 2] == kMaskedScore) x23.x = -INFINITY;
+      if (s[4 * q + 3] == kMaskedScore) x23.y = -INFINITY;
     }
-    sum += (p[0] + p[1]) + (p[2] + p[3]);
-    w[q] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
+    const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+    const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+    sum2 = fadd2(sum2, fadd2(p01, p23));
+    w[q] = __byte_perm(cvt_e4m3x2(p01.x, p01.y), cvt_e4m3x2(p23.x, p23.y), 0x5410);
   }
   *reinterpret_cast<uint4 *>(prow + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   *reinterpret_cast<uint4 *>(prow + (((c16 + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
-  return sum;
 }
 
 template <int D, bool CAUSAL, typename OutT>
@@ -345,19 +367,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld_32x32b_x32(s_tmem + ch * 32, s);
         tmem_ld_wait(s);
         if (masked) mask_chunk(s, j * kTile + ch * 32, N, CAUSAL, row_g);
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) smax = max(smax, max(static_cast<int>(s[i]), static_cast<int>(s[i + 1])));
+        smax = max(smax, tree_max32(s));
       }
       const float c = cq * sk[j];
       const float m_new = fmaxf(m_ref, static_cast<float>(smax) * c);
       const float alpha = ex2_approx(m_ref - m_new);    // 0 at the first tile (m_ref = -inf)
-      const float moff = m_new - kLog2_448;
+      const float bconst = fmaf(kMagicF, c, m_new - kLog2_448);
 
       // pass 2: P~ -> E4M3 into P buffer (j & 1), once P V of tile j-2 has read it
       const int pb = x * 2 + (j & 1);
       if (!mbar_wait(&pv_done[pb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       uint8_t *prow = p_base + (j & 1) * L::kPBytes;
-      float tsum = 0.f;
+      float2 tsum2 = make_float2(0.f, 0.f);
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t s[32];
@@ -365,14 +386,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld_wait(s);
         if (masked) {
           mask_chunk(s, j * kTile + ch * 32, N, CAUSAL, row_g);
-          tsum += p_chunk<true>(s, c, moff, prow, ch * 2, r);
+          p_chunk<true>(s, c, bconst, prow, ch * 2, r, tsum2);
         } else {
-          tsum += p_chunk<false>(s, c, moff, prow, ch * 2, r);
+          p_chunk<false>(s, c, bconst, prow, ch * 2, r, tsum2);
         }
       }
+      const float tsum = tsum2.x + tsum2.y;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[x]);            // S_x may be overwritten by Q_x K_{j+1}^T
+      if (lane == 0) mbar_arrive(&s_free[x]);
       l448 = fmaf(alpha, l448, tsum);
 
       // two-level accumulation: flush O_in at a group start, or rescale on a max increase
