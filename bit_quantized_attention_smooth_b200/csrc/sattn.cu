@@ -11,7 +11,9 @@
 
 #include "../../include/sattn.h"
 #include "attn_i8f8.cuh"
+#include "attn_nvfp4.cuh"
 #include "quant_i8f8.cuh"
+#include "quant_nvfp4.cuh"
 
 namespace sattn {
 namespace {
@@ -32,13 +34,36 @@ int check_shape(int B, int H, int N, int d, int mode) {
   if (d != 64 && d != 128) return SATTN_ERR_UNSUPPORTED;
   const long long total = static_cast<long long>(B) * H * N * d;
   if (total >= (1LL << 31) || static_cast<long long>(B) * H >= 65536) return SATTN_ERR_UNSUPPORTED;
-  if ((mode & ~SATTN_FP16_IO) == SATTN_NVFP4) return SATTN_ERR_UNSUPPORTED;
   return SATTN_OK;
 }
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-sattn_ws_layout_t make_layout(int B, int H, int N, int d) {
+bool is_nvfp4(int mode) { return (mode & ~SATTN_FP16_IO) == SATTN_NVFP4; }
+
+// NVFP4 workspace: q8/k8/vt8 hold the packed E2M1 codes of Q, K - mean and
+// V^T (N rounded up to 32 tokens), sq/sk/sv the E4M3 scale blocks of Q, K, V.
+sattn_ws_layout_t make_layout_nvfp4(int B, int H, int N, int d) {
+  sattn_ws_layout_t L;
+  std::memset(&L, 0xFF, sizeof(L));
+  const size_t BH = static_cast<size_t>(B) * H;
+  L.nblk = (N + kBlockTokens - 1) / kBlockTokens;
+  L.nv = (N + 31) / 32 * 32;
+  size_t off = 0;
+  L.q8 = off;   off = align_up(off + BH * N * d / 2, kSectionAlign);
+  L.k8 = off;   off = align_up(off + BH * N * d / 2, kSectionAlign);
+  L.vt8 = off;  off = align_up(off + BH * d * L.nv / 2, kSectionAlign);
+  L.sq = off;   off = align_up(off + BH * L.nblk * (d / 64) * 512, kSectionAlign);
+  L.sk = off;   off = align_up(off + BH * L.nblk * (d / 64) * 512, kSectionAlign);
+  L.sv = off;   off = align_up(off + BH * L.nblk * 1024, kSectionAlign);
+  L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
+  L.ksum = off; off += BH * d * sizeof(double);
+  L.vmax = off; off = align_up(off + BH * d * sizeof(unsigned), kSectionAlign);
+  L.total = off;
+  return L;
+}
+
+sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d) {
   sattn_ws_layout_t L;
   std::memset(&L, 0xFF, sizeof(L));
   const size_t BH = static_cast<size_t>(B) * H;
@@ -56,6 +81,10 @@ sattn_ws_layout_t make_layout(int B, int H, int N, int d) {
   L.vmax = off; off = align_up(off + BH * d * sizeof(unsigned), kSectionAlign);
   L.total = off;
   return L;
+}
+
+sattn_ws_layout_t make_layout(int B, int H, int N, int d, int mode) {
+  return is_nvfp4(mode) ? make_layout_nvfp4(B, H, N, d) : make_layout_i8f8(B, H, N, d);
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -111,6 +140,55 @@ int launch_quant_i8f8(const void *q, const void *k, const void *v, int BH, int N
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
+template <typename T, int D>
+int launch_quant_nvfp4(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws,
+                       const sattn_ws_layout_t &L, cudaStream_t st) {
+  double *ksum = reinterpret_cast<double *>(ws + L.ksum);
+  unsigned *vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
+  if (cudaMemsetAsync(ws + L.ksum, 0, L.total - L.ksum, st) != cudaSuccess) return SATTN_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.sv, 0, static_cast<size_t>(BH) * L.nblk * 1024, st) != cudaSuccess) return SATTN_ERR_CUDA;
+  const int tpc = 512;
+  kv_stats_kernel<T, D><<<dim3((N + tpc - 1) / tpc, BH), kQuantThreads, 0, st>>>(
+      static_cast<const T *>(k), static_cast<const T *>(v), ksum, vmax, N, tpc);
+  const dim3 grid(L.nblk, BH);
+  quant_rows_nvfp4_kernel<T, D, false><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(q), ws + L.q8, ws + L.sq,
+                                                                       nullptr, nullptr, N);
+  quant_rows_nvfp4_kernel<T, D, true><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(k), ws + L.k8, ws + L.sk,
+                                                                      ksum, reinterpret_cast<float *>(ws + L.mu), N);
+  quant_v_nvfp4_kernel<T, D><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(v), ws + L.vt8, ws + L.sv, N, L.nv);
+  return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, typename OutT>
+int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
+                      cudaStream_t st) {
+  using SL = AttnF4Smem<D>;
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle swqk = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  const uint64_t rowb = D / 2;
+  if (!make_map_u8(&tq, ws + L.q8, rowb, N, BH, rowb, static_cast<uint64_t>(N) * rowb, rowb, kTile, swqk) ||
+      !make_map_u8(&tk, ws + L.k8, rowb, N, BH, rowb, static_cast<uint64_t>(N) * rowb, rowb, kTile, swqk) ||
+      !make_map_u8(&tv, ws + L.vt8, (N + 1) / 2, D, BH, L.nv / 2, static_cast<uint64_t>(L.nv / 2) * D, kTile / 2, D,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return SATTN_ERR_CUDA;
+  // More than half of the SM's shared memory: one CTA (and its 512 TMEM
+  // columns) per SM.
+  const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
+  auto kern = attn_nvfp4_kernel<D, CAUSAL, OutT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SATTN_ERR_CUDA;
+  AttnF4Args a;
+  a.sfq = ws + L.sq;
+  a.sfk = ws + L.sk;
+  a.sfv = ws + L.sv;
+  a.out = out;
+  a.N = N;
+  a.nblk = L.nblk;
+  a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  kern<<<dim3(L.nblk, BH), kF4Threads, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+}
+
 template <int D, bool CAUSAL, typename OutT>
 int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
                      cudaStream_t st) {
@@ -147,7 +225,10 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
 
 template <int D, typename OutT>
 int dispatch_attn(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, int causal, float sm,
-                  cudaStream_t st) {
+                  bool nvfp4, cudaStream_t st) {
+  if (nvfp4)
+    return causal ? launch_attn_nvfp4<D, true, OutT>(ws, L, out, BH, N, sm, st)
+                  : launch_attn_nvfp4<D, false, OutT>(ws, L, out, BH, N, sm, st);
   return causal ? launch_attn_i8f8<D, true, OutT>(ws, L, out, BH, N, sm, st)
                 : launch_attn_i8f8<D, false, OutT>(ws, L, out, BH, N, sm, st);
 }
@@ -169,14 +250,14 @@ extern "C" {
 
 size_t sattn_workspace_bytes(int B, int H, int N, int d, int mode) {
   if (check_shape(B, H, N, d, mode) != SATTN_OK) return 0;
-  return make_layout(B, H, N, d).total;
+  return make_layout(B, H, N, d, mode).total;
 }
 
 int sattn_workspace_layout(int B, int H, int N, int d, int mode, sattn_ws_layout_t *out) {
   if (out == nullptr) return SATTN_ERR_INVALID_ARG;
   const int st = check_shape(B, H, N, d, mode);
   if (st != SATTN_OK) return st;
-  *out = make_layout(B, H, N, d);
+  *out = make_layout(B, H, N, d, mode);
   return SATTN_OK;
 }
 
@@ -186,12 +267,19 @@ int sattn_quantize(const void *q, const void *k, const void *v, int B, int H, in
   if (st != SATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SATTN_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
-  const sattn_ws_layout_t L = make_layout(B, H, N, d);
+  const sattn_ws_layout_t L = make_layout(B, H, N, d, mode);
   if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const int BH = B * H;
   const bool fp16 = (mode & SATTN_FP16_IO) != 0;
+  if (is_nvfp4(mode)) {
+    if (d == 128)
+      return fp16 ? launch_quant_nvfp4<__half, 128>(q, k, v, BH, N, ws, L, cs)
+                  : launch_quant_nvfp4<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, cs);
+    return fp16 ? launch_quant_nvfp4<__half, 64>(q, k, v, BH, N, ws, L, cs)
+                : launch_quant_nvfp4<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, cs);
+  }
   if (d == 128)
     return fp16 ? launch_quant_i8f8<__half, 128>(q, k, v, BH, N, ws, L, cs)
                 : launch_quant_i8f8<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, cs);
@@ -205,7 +293,7 @@ int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B
   if (st != SATTN_OK) return st;
   if (!aligned16(out)) return SATTN_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
-  const sattn_ws_layout_t L = make_layout(B, H, N, d);
+  const sattn_ws_layout_t L = make_layout(B, H, N, d, mode);
   if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
   const uint8_t *ws = static_cast<const uint8_t *>(workspace);
   if (static_cast<const uint8_t *>(out) < ws + L.total &&
@@ -215,11 +303,12 @@ int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * H;
   const bool fp16 = (mode & SATTN_FP16_IO) != 0;
+  const bool f4 = is_nvfp4(mode);
   if (d == 128)
-    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, cs)
-                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, cs);
-  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, cs)
-              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, cs);
+    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, f4, cs)
+                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, f4, cs);
+  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, f4, cs)
+              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, f4, cs);
 }
 
 int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
@@ -235,7 +324,7 @@ int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int
   }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SATTN_ERR_CUDA;
-  const size_t need = make_layout(B, H, N, d).total;
+  const size_t need = make_layout(B, H, N, d, mode).total;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   void *ws = nullptr;
   size_t ws_bytes = 0;
@@ -315,7 +404,7 @@ extern "C" int sattn_fwd_noalloc(const void *q, const void *k, const void *v, vo
     const uint8_t *p = static_cast<const uint8_t *>(in);
     if (o < p + io_bytes && p < o + io_bytes) return SATTN_ERR_INVALID_ARG;
   }
-  const size_t need = make_layout(B, H, N, d).total;
+  const size_t need = make_layout(B, H, N, d, mode).total;
   if (need > SATTN_NOALLOC_MAX_BYTES) return SATTN_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SATTN_ERR_CUDA;

@@ -45,6 +45,16 @@ def test_status_strings(L):
     assert b"unknown" in L.sattn_status_string(99)
 
 
+def test_nvfp4_workspace_layout(L):
+    lay = sattn.workspace_layout(1, 12, 32760, 128, mode="nvfp4")
+    bh, n, d = 12, 32760, 128
+    assert lay["nv"] == 32768 and lay["nblk"] == 256
+    assert lay["k8"] - lay["q8"] >= bh * n * d // 2
+    assert lay["sk"] - lay["sq"] >= bh * 256 * 2 * 512
+    assert lay["mu"] - lay["sv"] >= bh * 256 * 1024
+    assert lay["total"] == L.sattn_workspace_bytes(1, 12, 32760, 128, NVFP4)
+
+
 def test_workspace_bytes_and_layout(L):
     assert L.sattn_workspace_bytes(1, 2, 256, 64, FP16) > 0
     assert L.sattn_workspace_bytes(1, 2, 0, 64, BF16) == 0       # N < 1
@@ -75,7 +85,8 @@ def test_invalid_arguments_rejected_before_launch(L):
     assert q(p, p, p, 1, 2, 256, 64, BF16, None, 1 << 30, None) == WORKSPACE
     assert q(p, p, p, 1, 2, 256, 64, BF16, ctypes.c_void_p((1 << 21) + 16), 1 << 30, None) == WORKSPACE
     assert q(p, p, p, 1, 2, 256, 64, BF16, ws, 16, None) == WORKSPACE
-    assert q(p, p, p, 1, 2, 256, 64, NVFP4, ws, 1 << 30, None) == UNSUPPORTED
+    assert q(p, p, p, 1, 2, 256, 64, NVFP4, ws, 16, None) == WORKSPACE       # rejected before any launch
+    assert q(p, p, p, 1, 2, 256, 96, NVFP4, ws, 1 << 30, None) == UNSUPPORTED
     assert q(p, p, p, 1 << 16, 1, 256, 64, BF16, ws, 1 << 40, None) == UNSUPPORTED   # B*H too large
     f = L.sattn_fwd_quantized
     assert f(ws, 1 << 30, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
