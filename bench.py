@@ -180,17 +180,33 @@ def run_gpu(args):
     q, k, v = W.make_inputs(w, dev)
     B, H, N, d = q.shape
     ops = w.ops()
-    workspace = torch.empty(sattn.workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    mode = args.mode
+    workspace = torch.empty(sattn.workspace_bytes(B, H, N, d, mode=mode), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        sattn.quantize(q, k, v, workspace=workspace)
+    def step(m=mode, ws=workspace):
+        sattn.quantize(q, k, v, mode=m, workspace=ws)
         ev_mid = torch.cuda.Event(enable_timing=True)
         ev_mid.record(stream)
-        sattn.fwd_quantized(workspace, (B, H, N, d), dtype=q.dtype, out=out)
+        sattn.fwd_quantized(ws, (B, H, N, d), mode=m, dtype=q.dtype, out=out)
         return ev_mid
+
+    def timed_steps(n, m=mode, ws=workspace):
+        """n device-timed steps with an L2 flush before each; returns (step ms list, attention ms list)."""
+        evs = []
+        for _ in range(n):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e2 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            e1 = step(m, ws)
+            e2.record(stream)
+            evs.append((e0, e1, e2))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(c) for a, b, c in evs], [b.elapsed_time(c) for a, b, c in evs], \
+            [a.elapsed_time(b) for a, b, c in evs]
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -215,21 +231,16 @@ def run_gpu(args):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    evs = []
-    for _ in range(args.steps):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e2 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        e1 = step()
-        e2.record(stream)
-        evs.append((e0, e1, e2))
-    torch.cuda.synchronize()
+    step_ms, attn_ms, quant_ms = timed_steps(args.steps)
     barrier()
     clocks = sampler.stop()
-    step_ms = [a.elapsed_time(c) for a, b, c in evs]
-    attn_ms = [b.elapsed_time(c) for a, b, c in evs]
-    quant_ms = [a.elapsed_time(b) for a, b, c in evs]
+    # the other mode on the same inputs (reported beside the headline mode)
+    other = "nvfp4" if mode == "i8f8" else "i8f8"
+    ws_other = torch.empty(sattn.workspace_bytes(B, H, N, d, mode=other), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step(other, ws_other)
+    o_step, o_attn, o_quant = timed_steps(args.steps, other, ws_other)
+    del ws_other
     ms = sum(step_ms) / len(step_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
     if ws_n > 1:
@@ -246,7 +257,7 @@ def run_gpu(args):
         dq.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
-        sattn.fwd(dq, dk, dv, out=out)
+        sattn.fwd(dq, dk, dv, out=out, mode=mode)
         hout.copy_(out, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -270,8 +281,17 @@ def run_gpu(args):
     line = None
     if rank == 0:
         peaks, src = measured_peaks()
-        peak_i8 = 2.0 * peaks["bf16_tflops"]          # INT8/FP8 dense = 2 x bf16 (nominal 4.5 / 2.25)
+        ratio = {"i8f8": 2.0, "nvfp4": 4.0}               # dense INT8/FP8 = 2 x bf16, FP4 = 4 x bf16 (nominal)
+        datasheet = {"i8f8": 4500.0, "nvfp4": 9000.0}
+        peak_i8 = ratio[mode] * peaks["bf16_tflops"]
         achieved = ops / (attn_avg * 1e-3) / 1e12
+        o_ms, o_attn_avg = sum(o_step) / len(o_step), sum(o_attn) / len(o_attn)
+        o_achieved = ops / (o_attn_avg * 1e-3) / 1e12
+        other_line = {"mode": other, "value": ops / (o_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": o_ms,
+                      "attention_kernel": {"ms": o_attn_avg, "tops": o_achieved,
+                                           "frac_of_datasheet": o_achieved / datasheet[other],
+                                           "frac_of_measured_peak": o_achieved / (ratio[other] * peaks["bf16_tflops"])},
+                      "quantize_ms": sum(o_quant) / len(o_quant)}
         traffic = None
         tpath = os.path.join(ROOT, "profiles", "attn_i8f8_traffic.json")
         if os.path.exists(tpath):
@@ -289,22 +309,27 @@ def run_gpu(args):
         line = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8 QK^T / e4m3 PV (fp32 softmax + accumulation)",
+            "vs_baseline": None,
+            "dtype": ("int8 QK^T / e4m3 PV (fp32 softmax + accumulation)" if mode == "i8f8"
+                      else "nvfp4 QK^T / nvfp4 PV (e2m1 + e4m3 block scales; fp32 softmax + accumulation)"),
             "data": "synthetic",
-            "config": {"workload": w.name, "mode": "I8QK_F8PV", "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+            "config": {"workload": w.name, "mode": "I8QK_F8PV" if mode == "i8f8" else "NVFP4", "B": w.B, "H": w.H,
+                       "N": w.N, "d": w.d,
                        "causal": False, "io_dtype": w.dtype, "parallelism": f"replicas x{ws_n} (independent heads)",
                        "l2": "flushed between steps (256 MiB write, outside the step events)"},
             "attention_kernel": {"ms": attn_avg, "tops": achieved,
-                                 "frac_of_datasheet_4500": achieved / 4500.0},
+                                 "frac_of_datasheet": achieved / datasheet[mode]},
+            "other_mode": other_line,
             "quantize_ms": sum(quant_ms) / len(quant_ms),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TFLOP/s",
                          "frac": achieved / peak_i8, "traffic": traffic,
-                         "peak_source": f"{src}: 2 x bf16 burst {peaks['bf16_tflops']} (INT8/FP8 dense ratio 2)"},
+                         "peak_source": f"{src}: {ratio[mode]:.0f} x bf16 burst {peaks['bf16_tflops']} "
+                                        f"(nominal dense ratio of {mode} to bf16)"},
             "cpu_baseline": cpu,
             "e2e": {"value": ws_n * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
                     "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                     "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e2e_ms},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": 5 * args.steps,   # per step: stats, quant Q, quant K, quant V, attention
             "clocks": clocks,
             "device_error_word": err,
         }
@@ -333,6 +358,7 @@ def main():
     ap.add_argument("--impl", default="sattn", choices=["sattn", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="i8f8", choices=["i8f8", "nvfp4"])
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps of the GPU path only (for ncu captures)")
     args = ap.parse_args()
