@@ -13,11 +13,17 @@
 //   O_out  = alpha O_out + s1 O_in  (every tile: s1 changes per tile),  l = alpha l + rowsum(P~)
 //   O      = O_out / l
 //
-// CTA = one 128-row query tile of one (b, h); 6 warps:
-//   warps 0-3  softmax / two-stage quantisation / flush / epilogue (row t = TMEM lane t)
-//   warp 4     TMA producer (codes by tensor maps, scale factors by 1-D bulk copies)
-//   warp 5     TMEM allocator and single-thread MMA issuer; it also moves the
+// CTA = one 128-row query tile of one (b, h); 10 warps:
+//   warps 0-3  softmax, left half: keys 0-63 of each key tile and output
+//              columns [0, D/2) of row 32 w + lane (TMEM lane quarter w)
+//   warps 4-7  softmax, right half: keys 64-127, output columns [D/2, D)
+//   warp 8     TMA producer (codes by tensor maps, scale factors by 1-D bulk copies)
+//   warp 9     TMEM allocator and single-thread MMA issuer; it also moves the
 //              scale factors from shared to tensor memory (tcgen05.cp 32x128b.warpx4)
+// The two threads of a row exchange their halves' maxima through shared
+// memory (a bounded two-warp mbarrier per lane quarter); each quantises its
+// 64 keys of P (exactly the 64-key slice of one block-scaled MMA) and keeps
+// its half of the outer accumulator in registers.
 // TMEM columns: S [0,128) [128,256), O_in [256,256+D), scale factors from 384.
 // Scale factors of a 128-row operand and a 64-value slice of the contraction
 // axis occupy 4 columns: row m at lane m % 32 of every sub-partition, column
@@ -33,7 +39,7 @@
 
 namespace sattn {
 
-constexpr int kF4Threads = 192;
+constexpr int kF4Threads = 320;
 constexpr float kLog2_2688 = 11.392317422778761f;   // log2(448 * 6)
 
 struct AttnF4Args {
@@ -64,10 +70,11 @@ struct AttnF4Smem {
   static constexpr int kSfK = kSfQ + kSfQK;
   static constexpr int kSfVo = kSfK + kKVStages * kSfQK;
   static constexpr int kSfPo = kSfVo + kKVStages * kSfV;
-  static constexpr int kBar = kSfPo + 2 * kSfP;
+  static constexpr int kX = kSfPo + 2 * kSfP;          // float [2 phases][2 halves][128] + [2][128]
+  static constexpr int kBar = kX + (2 * 2 * 128 + 2 * 128) * 4;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
-  // p_full[2], pv_done[2], drain
-  static constexpr int kNumBars = 1 + 4 * kKVStages + 8 + 1;
+  // p_full[2], pv_done[2], pair[4], drain
+  static constexpr int kNumBars = 1 + 4 * kKVStages + 8 + 4 + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 256;     // 256 bytes of slack after the last buffer
   static constexpr int kAlloc = kBytes + 1024;
@@ -151,7 +158,10 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   uint64_t *s_free = s_full + 2;            // [2]
   uint64_t *p_full = s_free + 2;            // [2]
   uint64_t *pv_done = p_full + 2;           // [2]
-  uint64_t *drain_bar = pv_done + 2;
+  uint64_t *pair = pv_done + 2;             // [lane quarter]
+  uint64_t *drain_bar = pair + 4;
+  float *xmax = reinterpret_cast<float *>(smem + L::kX);                  // [2][2][128]
+  float *xl = reinterpret_cast<float *>(smem + L::kX + 2 * 2 * 128 * 4);  // [2][128]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
@@ -165,11 +175,11 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                         : static_cast<int>(blockIdx.x);
   const int nkv = CAUSAL ? min(qt + 1, nkv_all) : nkv_all;
 
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (tid == 128) {
+  if (tid == 256) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(&k_full[s], 1);
@@ -179,15 +189,16 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_free[b], 8);   // one arrival per softmax warp
+      mbar_init(&p_full[b], 8);
       mbar_init(&pv_done[b], 1);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&pair[i], 2);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (tid == 160) {
+  if (tid == 288) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       int last_j = -1;
@@ -233,7 +244,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdQK = idesc_nvfp4(kTile, kTile);
@@ -299,14 +310,17 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax warps
-    const int r = tid;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    constexpr int kHalfD = D / 2;
+    const int h = warp >> 2;                          // half of the row
+    const int wq = warp & 3;                          // TMEM lane quarter
+    const int r = wq * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const int row_g = qt * kTile + r;
     const float cl = args.sm_log2;                    // S is already dequantised by the MMA
-    float o_out[D];
+    float o_out[kHalfD];
 #pragma unroll
-    for (int i = 0; i < D; ++i) o_out[i] = 0.f;
-    float m_ref = -INFINITY, l = 0.f;
+    for (int i = 0; i < kHalfD; ++i) o_out[i] = 0.f;
+    float m_ref = -INFINITY, l = 0.f;                 // l: this half's share of the row sum
     float a_pend = 0.f, s1_pend = 0.f;                // factors of the tile whose P V is pending
     bool ok = true;
 
@@ -314,101 +328,92 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       const int b = j & 1;
       if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t s_tmem = tmem + lane_base + b * kTile;
+      const uint32_t s_tmem = tmem + lane_base + b * kTile + h * 64;
+      uint32_t sa[32], sb[32];
+      tmem_ld_32x32b_x32(s_tmem, sa);
+      tmem_ld_32x32b_x32(s_tmem + 32, sb);
+      tmem_ld_wait(sa);
+      tmem_ld_wait(sb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[b]);          // S_b may take Q K_{j+2}^T
       const bool masked = ((j == nkv_all - 1) && (N & (kTile - 1))) || (CAUSAL && j == qt);
-
-      // pass 1: maxima of the eight 16-key blocks of the row
-      float bmax[8];
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sr[32];
-        tmem_ld_32x32b_x32(s_tmem + ch * 32, sr);
-        tmem_ld_wait(sr);
-        float m0 = -INFINITY, m1 = -INFINITY;
+      if (masked) {
+        const int kv0 = j * kTile + h * 64;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int kv = j * kTile + ch * 32 + i;
-          float sv = __uint_as_float(sr[i]);
-          if (masked && (kv >= N || (CAUSAL && kv > row_g))) sv = -INFINITY;
-          if (i < 16) m0 = fmaxf(m0, sv);
-          else m1 = fmaxf(m1, sv);
+          if (kv0 + i >= N || (CAUSAL && kv0 + i > row_g)) sa[i] = __float_as_uint(-INFINITY);
+          if (kv0 + 32 + i >= N || (CAUSAL && kv0 + 32 + i > row_g)) sb[i] = __float_as_uint(-INFINITY);
         }
-        // dynamic index into bmax is avoided: select by chunk
-#pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2)
-          if (c2 == ch) {
-            bmax[2 * c2] = m0;
-            bmax[2 * c2 + 1] = m1;
-          }
       }
-      float tmax = bmax[0];
+      // maxima of the four 16-key blocks of this half, then the row max via the partner
+      float bmax[4];
 #pragma unroll
-      for (int i = 1; i < 8; ++i) tmax = fmaxf(tmax, bmax[i]);
+      for (int q = 0; q < 2; ++q) {
+        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          m0 = fmaxf(m0, __uint_as_float(q == 0 ? sa[i] : sb[i]));
+          m1 = fmaxf(m1, __uint_as_float(q == 0 ? sa[16 + i] : sb[16 + i]));
+        }
+        bmax[2 * q] = m0;
+        bmax[2 * q + 1] = m1;
+      }
+      const float hmax = fmaxf(fmaxf(bmax[0], bmax[1]), fmaxf(bmax[2], bmax[3]));
+      xmax[((j & 1) * 2 + h) * 128 + r] = hmax;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pair[wq]);
+      if (!mbar_wait(&pair[wq], j & 1, abort_flag)) { ok = false; break; }
+      const float tmax = fmaxf(hmax, xmax[((j & 1) * 2 + (1 - h)) * 128 + r]);
       const float m_tile = tmax * cl;                   // finite: every processed tile has a valid key
       const float m_new = fmaxf(m_ref, m_tile);
       const float alpha = ex2_approx(m_ref - m_new);
       const float s1 = ex2_approx(m_tile - m_new) * (1.f / 2688.f);
       const float moff = m_tile - kLog2_2688;           // P2 = 2^(S2 - moff) <= 2688
 
-      // pass 2: two-stage NVFP4 quantisation of P into buffer b
+      // two-stage NVFP4 quantisation of this half of P into buffer b (key slice h)
       if (!mbar_wait(&pv_done[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       uint8_t *prow = smem + L::kP + b * L::kPBytes + r * 64;
-      uint8_t *psf = smem + L::kSfPo + b * L::kSfP;
+      uint8_t *psf = smem + L::kSfPo + b * L::kSfP + h * 512;
       float psum = 0.f;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t sr[32];
-        tmem_ld_32x32b_x32(s_tmem + ch * 32, sr);
-        tmem_ld_wait(sr);
-        float bm0 = 0.f, bm1 = 0.f;
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2)
-          if (c2 == ch) {
-            bm0 = bmax[2 * c2];
-            bm1 = bmax[2 * c2 + 1];
-          }
+      for (int q = 0; q < 2; ++q) {
         uint32_t w[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float amax = ex2_approx(fmaf(h == 0 ? bm0 : bm1, cl, -moff));
+        for (int hb = 0; hb < 2; ++hb) {
+          const int blk = 2 * q + hb;                     // 16-key block within this half
+          const float amax = ex2_approx(fmaf(bmax[blk], cl, -moff));
           const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
           const float sc = e4m3_to_float(sc_code);
           const float inv = sc > 0.f ? 1.f / sc : 0.f;
-          const int blk = ch * 2 + h;
-          psf[(blk >> 2) * 512 + sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
+          psf[sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
           uint32_t packed[2] = {0u, 0u};
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
-            const int kv = j * kTile + ch * 32 + h * 16 + i;
-            float x0 = fmaf(__uint_as_float(sr[h * 16 + i]), cl, -moff);
-            float x1 = fmaf(__uint_as_float(sr[h * 16 + i + 1]), cl, -moff);
-            if (masked) {
-              if (kv >= N || (CAUSAL && kv > row_g)) x0 = -INFINITY;
-              if (kv + 1 >= N || (CAUSAL && kv + 1 > row_g)) x1 = -INFINITY;
-            }
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const uint32_t v0 = q == 0 ? sa[hb * 16 + i] : sb[hb * 16 + i];
+            const uint32_t v1 = q == 0 ? sa[hb * 16 + i + 1] : sb[hb * 16 + i + 1];
+            const float p0 = ex2_approx(fmaf(__uint_as_float(v0), cl, -moff));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(v1), cl, -moff));
             psum += p0 + p1;
             packed[i >> 3] |= cvt_e2m1x2(p0 * inv, p1 * inv) << (4 * (i & 7));
           }
-          w[2 * h] = packed[0];
-          w[2 * h + 1] = packed[1];
+          w[2 * hb] = packed[0];
+          w[2 * hb + 1] = packed[1];
         }
-        // 16 bytes = keys ch*32 .. ch*32+31; 64-byte swizzled K-major row
-        *reinterpret_cast<uint4 *>(prow + ((ch ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        // 16 bytes = keys h*64 + q*32 .. +31; 64-byte swizzled K-major row
+        const int c16 = h * 2 + q;
+        *reinterpret_cast<uint4 *>(prow + ((c16 ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[b]);
 
-      // flush the previous tile: O_out = a O_out + s1 O_in
+      // flush the previous tile: O_out = a O_out + s1 O_in (this half of the columns)
       if (j > 0) {
         const int t = j - 1;
         if (!mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 0; ch < kHalfD / 32; ++ch) {
           uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + ch * 32, o);
+          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + ch * 32, o);
           tmem_ld_wait(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o_out[ch * 32 + i] = fmaf(a_pend, o_out[ch * 32 + i], s1_pend * __uint_as_float(o[i]));
@@ -426,15 +431,18 @@ __global__ void __launch_bounds__(kF4Threads, 1)
 
     // ---------------------------------------------------------- epilogue
     if (ok && nkv > 0) {
+      xl[h * 128 + r] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pair[wq]);
       const int t = nkv - 1;
-      if (mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) {
+      if (mbar_wait(&pair[wq], nkv & 1, abort_flag) && mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) {
         tc_fence_after();
-        const float inv_l = 1.f / l;
-        OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D;
+        const float inv_l = 1.f / (xl[r] + xl[128 + r]);
+        OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D + h * kHalfD;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 0; ch < kHalfD / 32; ++ch) {
           uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + ch * 32, o);
+          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + ch * 32, o);
           tmem_ld_wait(o);
           uint32_t packed[16];
 #pragma unroll
@@ -456,7 +464,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
