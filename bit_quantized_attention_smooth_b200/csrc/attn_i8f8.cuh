@@ -12,9 +12,10 @@
 // Two-level accumulation: the tensor cores accumulate O_in over a group of
 // kFlushEvery key tiles; at the start of every group the softmax threads add
 // O_in into the outer FP32 accumulator O_out (registers) and the next P V
-// overwrites O_in.  When a row's running max grows inside a group, that row's
-// O_in and O_out are rescaled by alpha = 2^(m_old - m_new) (per warp, only
-// when some lane of the warp needs it).  Both happen after P of the tile has
+// overwrites O_in.  When a row's running max grows, O_out is rescaled by
+// alpha = 2^(m_old - m_new) through a per-row factor (O_out = beta * o_out,
+// beta *= alpha), and inside a group that row's O_in in TMEM is multiplied by
+// alpha (per warp, only when some lane of the warp needs it).  Both happen after P of the tile has
 // been written, when the previous P V has long completed.  Finally
 //   O = (O_out + O_in) * s_v[c] / (448 l).
 //
@@ -351,6 +352,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < D; ++i) o_out[i] = 0.f;
     float m_ref = -INFINITY;
     float l448 = 0.f;          // sum of 448 * P~ (the static FP8 scale folded in)
+    float beta = 1.f;          // the outer accumulator is beta * o_out (rescaled lazily)
     bool ok = true;
 
     for (int j = 0; j < nkv; ++j) {
@@ -404,25 +406,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = j - 1;
         if (!mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        if (boundary) {
+          // O_out += O_in (both relative to m_ref); o_out holds O_out / beta
+          const float inv_beta = 1.f / beta;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
-          tmem_ld_wait(o);
-          if (boundary) {
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
+            tmem_ld_wait(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              o_out[ch * 32 + i] = alpha * (o_out[ch * 32 + i] + __uint_as_float(o[i]));
-          } else {
+            for (int i = 0; i < 32; ++i) o_out[ch * 32 + i] = fmaf(__uint_as_float(o[i]), inv_beta, o_out[ch * 32 + i]);
+          }
+        } else {
+          // the group's partial sum in TMEM must follow the new reference max
+#pragma unroll 1
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
+            tmem_ld_wait(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              o_out[ch * 32 + i] *= alpha;
-              o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            }
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st_32x32b_x32(o_tmem + ch * 32, o);
           }
+          tmem_st_wait();
         }
-        if (!boundary) tmem_st_wait();
+      }
+      beta *= alpha;
+      if (__any_sync(0xffffffffu, beta < 0x1p-64f)) {
+        // keep beta away from the float32 underflow range (rare)
+#pragma unroll
+        for (int i = 0; i < D; ++i) o_out[i] *= beta;
+        beta = 1.f;
       }
       fence_proxy_async_smem();                          // P writes -> async proxy (MMA)
       tc_fence_before();
@@ -447,8 +461,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float o0 = (o_out[ch * 32 + i] + __uint_as_float(o[i])) * sv[ch * 32 + i] * inv_l;
-            const float o1 = (o_out[ch * 32 + i + 1] + __uint_as_float(o[i + 1])) * sv[ch * 32 + i + 1] * inv_l;
+            const float o0 = fmaf(beta, o_out[ch * 32 + i], __uint_as_float(o[i])) * sv[ch * 32 + i] * inv_l;
+            const float o1 = fmaf(beta, o_out[ch * 32 + i + 1], __uint_as_float(o[i + 1])) * sv[ch * 32 + i + 1] * inv_l;
             packed[i >> 1] = pack2_out<OutT>(o0, o1);
           }
           if (row_g < N) {
