@@ -376,6 +376,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       uint8_t *prow = smem + L::kP + b * L::kPBytes + r * 64;
       uint8_t *psf = smem + L::kSfPo + b * L::kSfP + h * 512;
       float psum = 0.f;
+      const float2 cl2 = make_float2(cl, cl);
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         uint32_t w[4];
@@ -385,20 +386,33 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           const float amax = ex2_approx(fmaf(bmax[blk], cl, -moff));
           const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
           const float sc = e4m3_to_float(sc_code);
-          const float inv = sc > 0.f ? 1.f / sc : 0.f;
           psf[sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
-          uint32_t packed[2] = {0u, 0u};
+          // P2 / scale = 2^(S2 - moff - log2 scale): the division folds into the
+          // exponent's constant; the block's P2 sum is scale * sum(P2 / scale).
+          const bool live = sc > 0.f;
+          const float lsc = live ? __log2f(sc) : 0.f;
+          const float2 nb2 = make_float2(-(moff + lsc), -(moff + lsc));
+          float2 bsum = make_float2(0.f, 0.f);
+          uint32_t bytes[8];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
             const uint32_t v0 = q == 0 ? sa[hb * 16 + i] : sb[hb * 16 + i];
             const uint32_t v1 = q == 0 ? sa[hb * 16 + i + 1] : sb[hb * 16 + i + 1];
-            const float p0 = ex2_approx(fmaf(__uint_as_float(v0), cl, -moff));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(v1), cl, -moff));
-            psum += p0 + p1;
-            packed[i >> 3] |= cvt_e2m1x2(p0 * inv, p1 * inv) << (4 * (i & 7));
+            const float2 x = ffma2(make_float2(__uint_as_float(v0), __uint_as_float(v1)), cl2, nb2);
+            const float2 y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            bsum = fadd2(bsum, y);
+            bytes[i >> 1] = cvt_e2m1x2(y.x, y.y);
           }
-          w[2 * hb] = packed[0];
-          w[2 * hb + 1] = packed[1];
+          if (live) psum = fmaf(sc, bsum.x + bsum.y, psum);
+          else {
+            // a block whose scale rounds to 0 has all-zero codes; its P2 values
+            // (below 6 * 2^-10 of 2688) still count towards the row sum
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bytes[i] = 0u;
+            psum += (bsum.x + bsum.y);
+          }
+          w[2 * hb] = __byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040), __byte_perm(bytes[2], bytes[3], 0x0040), 0x5410);
+          w[2 * hb + 1] = __byte_perm(__byte_perm(bytes[4], bytes[5], 0x0040), __byte_perm(bytes[6], bytes[7], 0x0040), 0x5410);
         }
         // 16 bytes = keys h*64 + q*32 .. +31; 64-byte swizzled K-major row
         const int c16 = h * 2 + q;
