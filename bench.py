@@ -45,6 +45,24 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def max_over_ranks(values, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (identity with one rank).
+
+    Device-timed step times are combined this way: the job's time is the slowest
+    rank's.  Works with gloo (CPU tensors) and NCCL (CUDA tensors)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(ops_per_rank, world, ms_max):
+    """Whole-job TOPS: operations of all ranks over the slowest rank's time."""
+    return world * ops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -243,10 +261,7 @@ def run_gpu(args):
     del ws_other
     ms = sum(step_ms) / len(step_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
-    if ws_n > 1:
-        t = torch.tensor([ms, attn_avg], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, attn_avg = t.tolist()
+    ms, attn_avg = max_over_ranks([ms, attn_avg], dev)
 
     # ---- end to end through the public call with host buffers (pinned)
     hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
@@ -271,11 +286,7 @@ def run_gpu(args):
         e2e_step()
     e_end.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end) / args.steps
-    if ws_n > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks([e_start.elapsed_time(e_end) / args.steps], dev)[0]
     err = sattn.device_error()
 
     line = None
@@ -305,7 +316,7 @@ def run_gpu(args):
             cpu = {"value": cpu_ops / cpu_s / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
                    "sample": f"head 0 of {w.H}, {rows_n} query rows x {w.N} keys, full-head quantisation "
                              f"included ({cpu_s:.1f} s); numpy float64 BLAS"}
-        value = ws_n * ops / (ms * 1e-3) / 1e12
+        value = job_throughput(ops, ws_n, ms)
         line = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -326,7 +337,7 @@ def run_gpu(args):
                          "peak_source": f"{src}: {ratio[mode]:.0f} x bf16 burst {peaks['bf16_tflops']} "
                                         f"(nominal dense ratio of {mode} to bf16)"},
             "cpu_baseline": cpu,
-            "e2e": {"value": ws_n * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+            "e2e": {"value": job_throughput(ops, ws_n, e2e_ms), "unit": "TOPS",
                     "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                     "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e2e_ms},
             "gpu_launches": 5 * args.steps,   # per step: stats, quant Q, quant K, quant V, attention
