@@ -22,8 +22,9 @@
  *   SATTN_NVFP4     : FP4 E2M1 values with one E4M3 scale per 16 values for
  *                     Q, K (along channels) and V (along tokens); P quantized
  *                     in two stages (a per-row, per-key-block float32 scale,
- *                     then NVFP4).  [not yet implemented: returns
- *                     SATTN_ERR_UNSUPPORTED]
+ *                     then NVFP4).  P.V is flushed into the outer
+ *                     accumulator every key block, since the stage-1 scale
+ *                     changes per block.
  *
  * Tensor layout (all modes): q, k, v, out are contiguous [B, H, N, d] ("BHND"),
  * element type bf16 (default) or fp16 (mode | SATTN_FP16_IO); out has the
@@ -135,7 +136,18 @@ int sattn_device_error(int clear);
  *   I8QK_F8PV: q8  int8   [B*H, N, d]        k8 int8 [B*H, N, d]
  *              vt8 e4m3   [B*H, d, Nv]  (Nv = N rounded up to 16)
  *              sq, sk float32 [B*H, ceil(N/128)]   sv, mu float32 [B*H, d]
- *              ksum float64 [B*H, d], vmax uint32 [B*H, d] (scratch) */
+ *              ksum float64 [B*H, d], vmax uint32 [B*H, d] (scratch)
+ *   NVFP4 (same fields, other contents):
+ *              q8, k8 E2M1 codes, two per byte (low nibble = even channel)
+ *                        [B*H, N, d/2]
+ *              vt8 E2M1 codes of V transposed [B*H, d, Nv/2] (Nv = N
+ *                        rounded up to 32; low nibble = even token)
+ *              sq, sk E4M3 block scales [B*H, ceil(N/128), d/64, 512]; row m
+ *                        (token within the 128-token block) and 16-channel
+ *                        block b at byte 16*(m%32) + 4*(m/32) + b
+ *              sv E4M3 block scales of V [B*H, ceil(N/128), 2, 512]; same
+ *                        byte order with m = channel and b = 16-token block
+ *              mu float32 [B*H, d]; ksum, vmax scratch as above */
 typedef struct {
   size_t q8, k8, vt8, sq, sk, sv, mu, ksum, vmax, total;
   int nv, nblk;
