@@ -24,7 +24,8 @@ STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
 
 # Every entry point declared in include/sattn.h.
 EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
-           "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc")
+           "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc",
+           "sattn_fwd_host")
 
 
 class SattnError(RuntimeError):
@@ -66,6 +67,8 @@ def lib():
         L.sattn_workspace_layout.argtypes = [i, i, i, i, i, ctypes.POINTER(WsLayout)]
         L.sattn_fwd_noalloc.restype = i
         L.sattn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+        L.sattn_fwd_host.restype = i
+        L.sattn_fwd_host.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
         _lib = L
     return _lib
 
@@ -149,6 +152,31 @@ def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None
                            int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype),
                            _stream(stream)),
            "sattn_fwd")
+    return out
+
+
+def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None):
+    """``fwd`` on host (CPU) tensors: copies in, computes and copies out chunk by
+    chunk, overlapping the transfers with the compute.  Pinned tensors
+    (``tensor.pin_memory()``) let the copies run asynchronously.  The call is
+    ordered on the current CUDA stream (or ``stream``); ``out`` holds the result
+    once that stream has passed it, e.g. after ``torch.cuda.synchronize()``."""
+    for t in (q, k, v):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous host tensors [B, H, N, d]")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share the shape [B, H, N, d]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    B, H, N, d = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    elif out.is_cuda or not out.is_contiguous() or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must be a contiguous host tensor like q")
+    _check(lib().sattn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
+                                int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype),
+                                _stream(stream)),
+           "sattn_fwd_host")
     return out
 
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -344,6 +345,138 @@ int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int
   const int s1 = sattn_quantize(q, k, v, B, H, N, d, mode, ws, ws_bytes, stream);
   if (s1 != SATTN_OK) return s1;
   return sattn_fwd_quantized(ws, ws_bytes, out, B, H, N, d, causal, sm_scale, mode, stream);
+}
+
+// Pipelined forward over host buffers: chunks of heads are copied in on one
+// stream, quantized and attended on two compute streams in turn, and copied
+// out on a fourth, so that the PCIe transfers of one chunk overlap the
+// compute of its neighbours.  Heads are independent, so every chunk runs the
+// same kernels as sattn_fwd on a B = 1, H = heads-in-chunk problem and the
+// result is bit-identical to sattn_fwd.
+namespace {
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_comp[2] = {nullptr, nullptr};
+  cudaEvent_t ev_start = nullptr, ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr},
+              ev_out[2] = {nullptr, nullptr};
+  uint8_t *slot[2] = {nullptr, nullptr};   // device q, k, v, out of one chunk
+  size_t slot_bytes = 0;
+  uint8_t *ws[2] = {nullptr, nullptr};     // workspace of one chunk
+  size_t ws_bytes = 0;
+};
+std::mutex g_host_mutex;
+HostPipe g_host[kMaxDevices];
+
+// Chunks per call: enough to overlap the copies with the compute, few enough
+// that each chunk still fills the GPU.
+constexpr int kHostChunks = 4;
+constexpr size_t kHostSlotCap = size_t(1) << 30;   // device bytes of one slot at most
+
+bool host_pipe_init(HostPipe &p) {
+  if (p.ready) return true;
+  cudaStream_t *ss[4] = {&p.s_in, &p.s_out, &p.s_comp[0], &p.s_comp[1]};
+  for (cudaStream_t *s : ss)
+    if (cudaStreamCreateWithFlags(s, cudaStreamNonBlocking) != cudaSuccess) return false;
+  cudaEvent_t *es[7] = {&p.ev_start, &p.ev_in[0], &p.ev_in[1], &p.ev_comp[0], &p.ev_comp[1], &p.ev_out[0], &p.ev_out[1]};
+  for (cudaEvent_t *e : es)
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+  p.ready = true;
+  return true;
+}
+
+// Grows the slot and workspace buffers; waits for the pipe's streams first,
+// since the old buffers may still be in use by the previous call.
+bool host_pipe_reserve(HostPipe &p, size_t slot_bytes, size_t ws_bytes) {
+  if (p.slot_bytes >= slot_bytes && p.ws_bytes >= ws_bytes) return true;
+  for (cudaStream_t s : {p.s_in, p.s_out, p.s_comp[0], p.s_comp[1]})
+    if (cudaStreamSynchronize(s) != cudaSuccess) return false;
+  if (p.slot_bytes < slot_bytes) {
+    for (uint8_t *&b : p.slot) {
+      if (b != nullptr && cudaFree(b) != cudaSuccess) return false;
+      b = nullptr;
+    }
+    p.slot_bytes = 0;
+    for (uint8_t *&b : p.slot)
+      if (cudaMalloc(reinterpret_cast<void **>(&b), slot_bytes) != cudaSuccess) return false;
+    p.slot_bytes = slot_bytes;
+  }
+  if (p.ws_bytes < ws_bytes) {
+    for (uint8_t *&b : p.ws) {
+      if (b != nullptr && cudaFree(b) != cudaSuccess) return false;
+      b = nullptr;
+    }
+    p.ws_bytes = 0;
+    for (uint8_t *&b : p.ws)
+      if (cudaMalloc(reinterpret_cast<void **>(&b), ws_bytes) != cudaSuccess) return false;
+    p.ws_bytes = ws_bytes;
+  }
+  return true;
+}
+}  // namespace
+
+int sattn_fwd_host(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
+                   float sm_scale, int mode, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return SATTN_ERR_INVALID_ARG;
+  const int BH = B * H;
+  const size_t head_bytes = static_cast<size_t>(N) * d * 2;
+  const size_t io_bytes = head_bytes * BH;
+  const uint8_t *o = static_cast<const uint8_t *>(out);
+  for (const void *in : {q, k, v}) {
+    const uint8_t *pi = static_cast<const uint8_t *>(in);
+    if (o < pi + io_bytes && pi < o + io_bytes) return SATTN_ERR_INVALID_ARG;
+  }
+  int hc = (BH + kHostChunks - 1) / kHostChunks;                       // heads per chunk
+  const int hc_cap = static_cast<int>(std::max<size_t>(1, kHostSlotCap / (4 * head_bytes)));
+  hc = std::max(1, std::min(hc, hc_cap));
+  const int nchunks = (BH + hc - 1) / hc;
+  const size_t part = align_up(head_bytes * hc, kSectionAlign);       // one of q, k, v, out in a slot
+  const size_t ws_need = make_layout(1, hc, N, d, mode).total;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SATTN_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_host_mutex);
+  HostPipe &p = g_host[dev];
+  if (!host_pipe_init(p) || !host_pipe_reserve(p, 4 * part, ws_need)) return SATTN_ERR_CUDA;
+  // everything this call does follows the caller's earlier work on its stream
+  if (cudaEventRecord(p.ev_start, cs) != cudaSuccess) return SATTN_ERR_CUDA;
+  for (cudaStream_t s : {p.s_in, p.s_out, p.s_comp[0], p.s_comp[1]})
+    if (cudaStreamWaitEvent(s, p.ev_start, 0) != cudaSuccess) return SATTN_ERR_CUDA;
+  const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k),
+                *hv = static_cast<const uint8_t *>(v);
+  uint8_t *hout = static_cast<uint8_t *>(out);
+  int last = 0;
+  for (int c = 0; c < nchunks; ++c) {
+    const int sl = c & 1;
+    const int h0 = c * hc, hn = std::min(hc, BH - h0);
+    const size_t off = head_bytes * h0, len = head_bytes * hn;
+    uint8_t *dq = p.slot[sl], *dk = dq + part, *dv = dk + part, *dout = dv + part;
+    // copy in, once compute of the chunk that last used this slot is done
+    if (cudaStreamWaitEvent(p.s_in, p.ev_comp[sl], 0) != cudaSuccess ||
+        cudaMemcpyAsync(dq, hq + off, len, cudaMemcpyHostToDevice, p.s_in) != cudaSuccess ||
+        cudaMemcpyAsync(dk, hk + off, len, cudaMemcpyHostToDevice, p.s_in) != cudaSuccess ||
+        cudaMemcpyAsync(dv, hv + off, len, cudaMemcpyHostToDevice, p.s_in) != cudaSuccess ||
+        cudaEventRecord(p.ev_in[sl], p.s_in) != cudaSuccess)
+      return SATTN_ERR_CUDA;
+    // compute, once the inputs are in and the slot's last output has been copied out
+    cudaStream_t sc = p.s_comp[sl];
+    if (cudaStreamWaitEvent(sc, p.ev_in[sl], 0) != cudaSuccess || cudaStreamWaitEvent(sc, p.ev_out[sl], 0) != cudaSuccess)
+      return SATTN_ERR_CUDA;
+    const sattn_stream_t ss = reinterpret_cast<sattn_stream_t>(sc);
+    int r = sattn_quantize(dq, dk, dv, 1, hn, N, d, mode, p.ws[sl], p.ws_bytes, ss);
+    if (r != SATTN_OK) return r;
+    r = sattn_fwd_quantized(p.ws[sl], p.ws_bytes, dout, 1, hn, N, d, causal, sm_scale, mode, ss);
+    if (r != SATTN_OK) return r;
+    // copy out
+    if (cudaEventRecord(p.ev_comp[sl], sc) != cudaSuccess || cudaStreamWaitEvent(p.s_out, p.ev_comp[sl], 0) != cudaSuccess ||
+        cudaMemcpyAsync(hout + off, dout, len, cudaMemcpyDeviceToHost, p.s_out) != cudaSuccess ||
+        cudaEventRecord(p.ev_out[sl], p.s_out) != cudaSuccess)
+      return SATTN_ERR_CUDA;
+    last = sl;
+  }
+  // the copies out run in order on one stream: the last one ends the call
+  return cudaStreamWaitEvent(cs, p.ev_out[last], 0) == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
 const char *sattn_status_string(int status) {

@@ -98,6 +98,27 @@ int sattn_fwd(const void *q, const void *k, const void *v, void *out,
               int B, int H, int N, int d, int causal, float sm_scale, int mode,
               sattn_stream_t stream);
 
+/* sattn_fwd on HOST buffers: q, k, v and out are host pointers ([B, H, N, d],
+ * same element type and layout as sattn_fwd); pinned (page-locked) memory lets
+ * the copies run asynchronously, pageable memory works but serializes them.
+ * The call splits the B*H heads into a few chunks and pipelines them: chunk c
+ * is copied to the device on one stream, quantized and attended on one of two
+ * compute streams, and copied back on a fourth stream, so that the PCIe
+ * transfers of one chunk overlap the compute of the others.  Attention heads
+ * are independent and every quantization scale is per head, so the output is
+ * bit-identical to sattn_fwd on the same inputs.  The device buffers (two
+ * chunks of q, k, v, out and two workspaces) and the streams are owned by the
+ * library, one set per device, created on first use with cudaMalloc and grown
+ * when a larger problem arrives (growing waits for the previous call's work).
+ * The call is ordered on `stream` like a kernel launch: its work starts after
+ * the work already queued on `stream`, and `out` holds the result once
+ * `stream` has passed the call (e.g. after cudaStreamSynchronize(stream)).
+ * q, k, v must stay unchanged and out untouched until then.  Calls on one
+ * device are serialized by the library.  `out` must not alias q, k or v. */
+int sattn_fwd_host(const void *q, const void *k, const void *v, void *out,
+                   int B, int H, int N, int d, int causal, float sm_scale, int mode,
+                   sattn_stream_t stream);
+
 /* Size of the static device workspace of sattn_fwd_noalloc: 64 MiB, enough
  * for B*H*N*d up to about 22 million elements (e.g. B=1, H=12, N=4096, d=128). */
 #define SATTN_NOALLOC_MAX_BYTES (64ull << 20)

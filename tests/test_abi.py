@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import bit_quantized_attention_smooth_b200 as sattn
 from bit_quantized_attention_smooth_b200 import build as sattn_build
@@ -97,3 +98,25 @@ def test_invalid_arguments_rejected_before_launch(L):
     assert g(p, p, p, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
     assert g(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
     assert g(p, p, p, mis, 1, 2, 256, 128, 0, 0.0, 0x200, None) == INVALID   # unknown flag
+
+
+def test_fwd_host_rejects_bad_arguments_before_any_cuda_call(L):
+    p = ctypes.c_void_p(1 << 20)          # host addresses, never dereferenced: validation fails first
+    o = ctypes.c_void_p(1 << 40)
+    h = L.sattn_fwd_host
+    assert h(None, p, p, o, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
+    assert h(p, p, p, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
+    assert h(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
+    assert h(p, p, p, o, 1, 2, 256, 96, 0, 0.0, BF16, None) == UNSUPPORTED
+    assert h(p, p, p, o, 1, 2, 0, 64, 0, 0.0, BF16, None) == INVALID
+    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, 0x200, None) == INVALID     # unknown flag
+
+
+def test_fwd_host_binding_rejects_device_or_mismatched_tensors():
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sattn.fwd_host(q, q, q[:, :1])
+    with pytest.raises(TypeError):
+        sattn.fwd_host(q, q, q.half())
+    with pytest.raises(ValueError):
+        sattn.fwd_host(q, q, q, out=torch.zeros(1, 2, 64, 32, dtype=torch.bfloat16))
