@@ -25,6 +25,9 @@ namespace sattn {
 
 constexpr int kBlockTokens = 128;   // quantisation block = attention tile height
 constexpr int kQuantThreads = 256;
+// Threads of the per-block quantizers: a block of 128 tokens is spread over
+// 512 threads so that each holds few values and an SM keeps more loads in flight.
+constexpr int kBlockQuantThreads = 512;
 
 template <typename T>
 __device__ __forceinline__ void load8(const T *p, float (&f)[8]);
@@ -79,6 +82,7 @@ __global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__rest
     acc[i] = 0.0;
     vm[i] = 0.f;
   }
+#pragma unroll 4
   for (int n = n_begin + r0; n < n_end; n += RPI) {
     float kf[8], vf[8];
     load8<T>(k + head + static_cast<size_t>(n) * D + cg * 8, kf);
@@ -108,7 +112,8 @@ __global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__rest
   }
 }
 
-__device__ __forceinline__ float block_max_256(float v, float *s_red) {
+template <int NT>
+__device__ __forceinline__ float block_max(float v, float *s_red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   const int warp = threadIdx.x >> 5;
@@ -116,22 +121,22 @@ __device__ __forceinline__ float block_max_256(float v, float *s_red) {
   __syncthreads();
   float m = s_red[0];
 #pragma unroll
-  for (int w = 1; w < kQuantThreads / 32; ++w) m = fmaxf(m, s_red[w]);
+  for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, s_red[w]);
   return m;
 }
 
 // Pass 2a: per-block INT8 of Q (IS_K = false) or of K - mu (IS_K = true).
-// grid (ceil(N/128), B*H), block 256.  Each thread owns a fixed group of 8
-// channels and (128 * D / 8) / 256 row positions.
+// grid (ceil(N/128), B*H), block kBlockQuantThreads.  Each thread owns a
+// fixed group of 8 channels and (128 * D / 8) / kBlockQuantThreads row positions.
 template <typename T, int D, bool IS_K>
-__global__ void __launch_bounds__(kQuantThreads) quant_qk_kernel(const T *__restrict__ x, int8_t *__restrict__ out,
+__global__ void __launch_bounds__(kBlockQuantThreads, 2) quant_qk_kernel(const T *__restrict__ x, int8_t *__restrict__ out,
                                                                  float *__restrict__ scale,
                                                                  const double *__restrict__ ksum,
                                                                  float *__restrict__ mu_out, int N, int nblk) {
   constexpr int LPR = D / 8;
-  constexpr int RPI = kQuantThreads / LPR;
+  constexpr int RPI = kBlockQuantThreads / LPR;
   constexpr int ITERS = kBlockTokens / RPI;
-  __shared__ float s_red[kQuantThreads / 32];
+  __shared__ float s_red[kBlockQuantThreads / 32];
 
   const int bh = blockIdx.y;
   const int blk = blockIdx.x;
@@ -139,10 +144,21 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qk_kernel(const T *__rest
   const int r0 = threadIdx.x / LPR;
   const size_t head = static_cast<size_t>(bh) * N * D;
 
-  float mu[8];
+  // every load first, so that the mean's float64 division below overlaps them
+  float val[ITERS][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) mu[i] = 0.f;
+  for (int it = 0; it < ITERS; ++it) {
+    const int n = blk * kBlockTokens + it * RPI + r0;
+    if (n < N) {
+      load8<T>(x + head + static_cast<size_t>(n) * D + cg * 8, val[it]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) val[it][i] = 0.f;
+    }
+  }
+  float amax = 0.f;
   if (IS_K) {
+    float mu[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       mu[i] = static_cast<float>(ksum[static_cast<size_t>(bh) * D + cg * 8 + i] / static_cast<double>(N));
@@ -150,26 +166,22 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qk_kernel(const T *__rest
 #pragma unroll
       for (int i = 0; i < 8; ++i) mu_out[static_cast<size_t>(bh) * D + cg * 8 + i] = mu[i];
     }
-  }
-
-  float val[ITERS][8];
-  float amax = 0.f;
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int n = blk * kBlockTokens + it * RPI + r0;
-    if (n < N) {
-      load8<T>(x + head + static_cast<size_t>(n) * D + cg * 8, val[it]);
+    for (int it = 0; it < ITERS; ++it) {
+      const bool valid = blk * kBlockTokens + it * RPI + r0 < N;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if (IS_K) val[it][i] = __fsub_rn(val[it][i], mu[i]);
+        val[it][i] = valid ? __fsub_rn(val[it][i], mu[i]) : 0.f;
         amax = fmaxf(amax, fabsf(val[it][i]));
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) val[it][i] = 0.f;
     }
+  } else {
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(val[it][i]));
   }
-  amax = block_max_256(amax, s_red);
+  amax = block_max<kBlockQuantThreads>(amax, s_red);
   const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
   if (threadIdx.x == 0) scale[static_cast<size_t>(bh) * nblk + blk] = s;
 
@@ -190,64 +202,70 @@ __global__ void __launch_bounds__(kQuantThreads) quant_qk_kernel(const T *__rest
 }
 
 // Pass 2b: per-channel FP8 E4M3 of V, stored transposed vt[bh][c][token]
-// with row length Nv (N rounded up to 16).  grid (ceil(N/128), B*H), block 256.
+// with row length Nv (N rounded up to 16).  grid (ceil(N/128), B*H), block
+// 4 D threads.  Thread t takes the 4 tokens 4 (t mod 32) .. + 3 of the block
+// and the 8 channels of group t / 32, packs the 4 codes of each channel into one word
+// (lowest token in the low byte), and the block is written out row by row:
+// every shared-memory access of a warp touches 32 consecutive words and every
+// global store is a full 128-byte row segment.
 template <typename T, int D>
-__global__ void __launch_bounds__(kQuantThreads) quant_v_kernel(const T *__restrict__ v, uint8_t *__restrict__ vt,
+__global__ void __launch_bounds__(4 * D, 2) quant_v_kernel(const T *__restrict__ v, uint8_t *__restrict__ vt,
                                                                 float *__restrict__ sv_out,
                                                                 const unsigned *__restrict__ vmax, int N,
                                                                 int Nv) {
-  constexpr int LPR = D / 8;
-  constexpr int RPI = kQuantThreads / LPR;
-  constexpr int ITERS = kBlockTokens / RPI;
-  constexpr int TROW = kBlockTokens + 16;  // padded smem row (bytes)
-  __shared__ __align__(16) uint8_t tile[D][TROW];
+  constexpr int CPT = 8;                     // channels per thread
+  constexpr int NT = 4 * D;                  // threads
+  constexpr int WPR = kBlockTokens / 4;      // words per channel row of the block (32)
+  __shared__ uint32_t tile[D][WPR];
 
   const int bh = blockIdx.y;
   const int blk = blockIdx.x;
-  const int cg = threadIdx.x % LPR;
-  const int r0 = threadIdx.x / LPR;
+  const int tq = threadIdx.x % WPR;          // token quad
+  const int c0 = (threadIdx.x / WPR) * CPT;  // first channel of this thread
   const size_t head = static_cast<size_t>(bh) * N * D;
 
-  float sv[8];
+  float sv[CPT];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float m = __uint_as_float(vmax[static_cast<size_t>(bh) * D + cg * 8 + i]);
+  for (int i = 0; i < CPT; ++i) {
+    const float m = __uint_as_float(vmax[static_cast<size_t>(bh) * D + c0 + i]);
     sv[i] = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
   }
-  if (blk == 0 && r0 == 0) {
+  if (blk == 0 && tq == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sv_out[static_cast<size_t>(bh) * D + cg * 8 + i] = sv[i];
+    for (int i = 0; i < CPT; ++i) sv_out[static_cast<size_t>(bh) * D + c0 + i] = sv[i];
   }
 
+  float f[4][CPT];
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int nl = it * RPI + r0;
-    const int n = blk * kBlockTokens + nl;
-    float f[8];
-    if (n < N) {
-      load8<T>(v + head + static_cast<size_t>(n) * D + cg * 8, f);
-    } else {
+  for (int r = 0; r < 4; ++r) {
+    const int n = blk * kBlockTokens + 4 * tq + r;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) f[i] = 0.f;
-    }
+    for (int g = 0; g < CPT; g += 8) {
+      float t8[8];
+      if (n < N) {
+        load8<T>(v + head + static_cast<size_t>(n) * D + c0 + g, t8);
+      } else {
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      const uint32_t two = cvt_e4m3x2(__fdiv_rn(f[i], sv[i]), __fdiv_rn(f[i + 1], sv[i + 1]));
-      tile[cg * 8 + i][nl] = static_cast<uint8_t>(two & 0xFFu);
-      tile[cg * 8 + i + 1][nl] = static_cast<uint8_t>(two >> 8);
+        for (int i = 0; i < 8; ++i) t8[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[r][g + i] = t8[i];
     }
   }
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f[0][i], sv[i]), __fdiv_rn(f[1][i], sv[i]));
+    const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f[2][i], sv[i]), __fdiv_rn(f[3][i], sv[i]));
+    tile[c0 + i][tq] = lo | (hi << 16);
+  }
   __syncthreads();
-  // D rows x 128 tokens = D * 8 chunks of 16 bytes.
   const int tok0 = blk * kBlockTokens;
-  const int valid_chunks = min(kBlockTokens, Nv - tok0) / 16;
-  for (int idx = threadIdx.x; idx < D * 8; idx += kQuantThreads) {
-    const int c = idx >> 3;
-    const int ch = idx & 7;
-    if (ch < valid_chunks) {
-      const uint4 u = *reinterpret_cast<const uint4 *>(&tile[c][ch * 16]);
-      *reinterpret_cast<uint4 *>(vt + (static_cast<size_t>(bh) * D + c) * Nv + tok0 + ch * 16) = u;
-    }
+  const int valid_words = min(kBlockTokens, Nv - tok0) / 4;
+  for (int idx = threadIdx.x; idx < D * WPR; idx += NT) {
+    const int c = idx / WPR;
+    const int w = idx % WPR;
+    if (w < valid_words)
+      *reinterpret_cast<uint32_t *>(vt + (static_cast<size_t>(bh) * D + c) * Nv + tok0 + 4 * w) = tile[c][w];
   }
 }
 

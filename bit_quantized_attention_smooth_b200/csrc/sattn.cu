@@ -130,13 +130,13 @@ int launch_quant_i8f8(const void *q, const void *k, const void *v, int BH, int N
   kv_stats_kernel<T, D><<<dim3((N + tpc - 1) / tpc, BH), kQuantThreads, 0, st>>>(
       static_cast<const T *>(k), static_cast<const T *>(v), ksum, vmax, N, tpc);
   const dim3 grid(L.nblk, BH);
-  quant_qk_kernel<T, D, false><<<grid, kQuantThreads, 0, st>>>(
+  quant_qk_kernel<T, D, false><<<grid, kBlockQuantThreads, 0, st>>>(
       static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq),
       nullptr, nullptr, N, L.nblk);
-  quant_qk_kernel<T, D, true><<<grid, kQuantThreads, 0, st>>>(
+  quant_qk_kernel<T, D, true><<<grid, kBlockQuantThreads, 0, st>>>(
       static_cast<const T *>(k), reinterpret_cast<int8_t *>(ws + L.k8), reinterpret_cast<float *>(ws + L.sk), ksum,
       reinterpret_cast<float *>(ws + L.mu), N, L.nblk);
-  quant_v_kernel<T, D><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(v), ws + L.vt8,
+  quant_v_kernel<T, D><<<grid, 4 * D, 0, st>>>(static_cast<const T *>(v), ws + L.vt8,
                                                         reinterpret_cast<float *>(ws + L.sv), vmax, N, L.nv);
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
