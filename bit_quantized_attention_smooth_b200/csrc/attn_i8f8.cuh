@@ -45,8 +45,8 @@ constexpr int kQTiles = 2;          // query tiles per CTA
 constexpr int kKVStages = 3;
 constexpr int kFlushEvery = 4;      // G: key tiles per inner accumulation group
 constexpr int kAttnThreads = 384;       // 3 warpgroups
-constexpr int kSoftmaxRegs = 216;       // per thread, softmax warpgroups 0 and 1
-constexpr int kControlRegs = 64;        // per thread, warpgroup 2 (TMA, MMA, 2 idle warps)
+constexpr int kSoftmaxRegs = 232;       // per thread, softmax warpgroups 0 and 1
+constexpr int kControlRegs = 40;        // per thread, warpgroup 2 (TMA, MMA, 2 idle warps)
 // setmaxnreg moves registers between warpgroups of the block; the split must
 // fit in what the block was launched with (threads x launch registers).
 constexpr int kRegsNeeded = 256 * kSoftmaxRegs + 128 * kControlRegs;
@@ -360,16 +360,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
       const bool masked = ((j == nkv_all - 1) && (N & (kTile - 1))) || (CAUSAL && j == qt);
 
-      // pass 1: row max of the integer scores (a rolled loop over 32-column
-      // chunks keeps the loop body small enough for the instruction cache)
+      // pass 1: row max of the integer scores (a rolled loop over two 64-column
+      // halves, each read with two loads behind one wait, keeps the loop body
+      // small enough for the instruction cache)
       int smax = INT_MIN;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t s[32];
-        tmem_ld_32x32b_x32(s_tmem + ch * 32, s);
-        tmem_ld_wait(s);
-        if (masked) mask_chunk(s, j * kTile + ch * 32, N, CAUSAL, row_g);
-        smax = max(smax, tree_max32(s));
+      for (int hh = 0; hh < 2; ++hh) {
+        // two 32-column loads behind one wait: one TMEM round trip per 64 columns
+        uint32_t s0[32], s1[32];
+        tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
+        tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
+        tmem_ld_wait(s0);
+        tmem_ld_wait(s1);
+        if (masked) {
+          mask_chunk(s0, j * kTile + hh * 64, N, CAUSAL, row_g);
+          mask_chunk(s1, j * kTile + hh * 64 + 32, N, CAUSAL, row_g);
+        }
+        smax = max(smax, max(tree_max32(s0), tree_max32(s1)));
       }
       const float c = cq * sk[j];
       const float m_new = fmaxf(m_ref, static_cast<float>(smax) * c);
@@ -382,15 +389,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint8_t *prow = p_base + (j & 1) * L::kPBytes;
       float2 tsum2 = make_float2(0.f, 0.f);
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t s[32];
-        tmem_ld_32x32b_x32(s_tmem + ch * 32, s);
-        tmem_ld_wait(s);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t s0[32], s1[32];
+        tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
+        tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
+        tmem_ld_wait(s0);
+        tmem_ld_wait(s1);
         if (masked) {
-          mask_chunk(s, j * kTile + ch * 32, N, CAUSAL, row_g);
-          p_chunk<true>(s, c, bconst, prow, ch * 2, r, tsum2);
+          mask_chunk(s0, j * kTile + hh * 64, N, CAUSAL, row_g);
+          mask_chunk(s1, j * kTile + hh * 64 + 32, N, CAUSAL, row_g);
+          p_chunk<true>(s0, c, bconst, prow, hh * 4, r, tsum2);
+          p_chunk<true>(s1, c, bconst, prow, hh * 4 + 2, r, tsum2);
         } else {
-          p_chunk<false>(s, c, bconst, prow, ch * 2, r, tsum2);
+          p_chunk<false>(s0, c, bconst, prow, hh * 4, r, tsum2);
+          p_chunk<false>(s1, c, bconst, prow, hh * 4 + 2, r, tsum2);
         }
       }
       const float tsum = tsum2.x + tsum2.y;
@@ -420,13 +432,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         } else {
           // the group's partial sum in TMEM must follow the new reference max
 #pragma unroll 1
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
-            tmem_ld_wait(o);
+          for (int ch = 0; ch < D / 32; ch += 2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld_32x32b_x32(o_tmem + ch * 32, o0);
+            tmem_ld_32x32b_x32(o_tmem + ch * 32 + 32, o1);
+            tmem_ld_wait(o0);
+            tmem_ld_wait(o1);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_32x32b_x32(o_tmem + ch * 32, o);
+            for (int i = 0; i < 32; ++i) {
+              o0[i] = __float_as_uint(__uint_as_float(o0[i]) * alpha);
+              o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+            }
+            tmem_st_32x32b_x32(o_tmem + ch * 32, o0);
+            tmem_st_32x32b_x32(o_tmem + ch * 32 + 32, o1);
           }
           tmem_st_wait();
         }
