@@ -422,12 +422,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // O_out += O_in (both relative to m_ref); o_out holds O_out / beta
           const float inv_beta = 1.f / beta;
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld_32x32b_x32(o_tmem + ch * 32, o);
-            tmem_ld_wait(o);
+          for (int ch = 0; ch < D / 32; ch += 2) {
+            uint32_t o0[32], o1[32];
+            tmem_ld_32x32b_x32(o_tmem + ch * 32, o0);
+            tmem_ld_32x32b_x32(o_tmem + ch * 32 + 32, o1);
+            tmem_ld_wait(o0);
+            tmem_ld_wait(o1);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o_out[ch * 32 + i] = fmaf(__uint_as_float(o[i]), inv_beta, o_out[ch * 32 + i]);
+            for (int i = 0; i < 32; ++i) {
+              o_out[ch * 32 + i] = fmaf(__uint_as_float(o0[i]), inv_beta, o_out[ch * 32 + i]);
+              o_out[ch * 32 + 32 + i] = fmaf(__uint_as_float(o1[i]), inv_beta, o_out[ch * 32 + 32 + i]);
+            }
           }
         } else {
           // the group's partial sum in TMEM must follow the new reference max

@@ -41,6 +41,7 @@ namespace sattn {
 
 constexpr int kF4Threads = 320;
 constexpr float kLog2_2688 = 11.392317422778761f;   // log2(448 * 6)
+constexpr float kLog2_6 = 2.584962500721156f;       // log2(6)
 
 struct AttnF4Args {
   const uint8_t *sfq;   // [BH][nblk][D/64][512]
@@ -370,6 +371,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       const float alpha = ex2_approx(m_ref - m_new);
       const float s1 = ex2_approx(m_tile - m_new) * (1.f / 2688.f);
       const float moff = m_tile - kLog2_2688;           // P2 = 2^(S2 - moff) <= 2688
+      const float moff6 = moff + kLog2_6;
 
       // two-stage NVFP4 quantisation of this half of P into buffer b (key slice h)
       if (!mbar_wait(&pv_done[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -383,8 +385,9 @@ __global__ void __launch_bounds__(kF4Threads, 1)
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
           const int blk = 2 * q + hb;                     // 16-key block within this half
-          const float amax = ex2_approx(fmaf(bmax[blk], cl, -moff));
-          const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
+          // scale = E4M3(block max of P2 / 6): the division by 6 folds into the exponent
+          const float amax6 = ex2_approx(fmaf(bmax[blk], cl, -moff6));
+          const uint32_t sc_code = cvt_e4m3x2(amax6, 0.f) & 0xFFu;
           const float sc = e4m3_to_float(sc_code);
           psf[sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
           // P2 / scale = 2^(S2 - moff - log2 scale): the division folds into the
@@ -424,13 +427,24 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         const int t = j - 1;
         if (!mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        if constexpr (kHalfD == 64) {
+          // both 32-column chunks behind one wait
+          uint32_t o0[32], o1[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD, o0);
+          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + 32, o1);
+          tmem_ld_wait(o0);
+          tmem_ld_wait(o1);
 #pragma unroll
-        for (int ch = 0; ch < kHalfD / 32; ++ch) {
+          for (int i = 0; i < 32; ++i) {
+            o_out[i] = fmaf(a_pend, o_out[i], s1_pend * __uint_as_float(o0[i]));
+            o_out[32 + i] = fmaf(a_pend, o_out[32 + i], s1_pend * __uint_as_float(o1[i]));
+          }
+        } else {
           uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + ch * 32, o);
+          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD, o);
           tmem_ld_wait(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o_out[ch * 32 + i] = fmaf(a_pend, o_out[ch * 32 + i], s1_pend * __uint_as_float(o[i]));
+          for (int i = 0; i < 32; ++i) o_out[i] = fmaf(a_pend, o_out[i], s1_pend * __uint_as_float(o[i]));
         }
       }
       l = fmaf(alpha, l, s1 * psum);
