@@ -350,15 +350,14 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       // maxima of the four 16-key blocks of this half, then the row max via the partner
       float bmax[4];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float m0 = -INFINITY, m1 = -INFINITY;
+      for (int blk = 0; blk < 4; ++blk) {
+        const uint32_t *v = (blk < 2 ? sa : sb) + (blk & 1) * 16;
+        float t[6];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          m0 = fmaxf(m0, __uint_as_float(q == 0 ? sa[i] : sb[i]));
-          m1 = fmaxf(m1, __uint_as_float(q == 0 ? sa[16 + i] : sb[16 + i]));
-        }
-        bmax[2 * q] = m0;
-        bmax[2 * q + 1] = m1;
+        for (int i = 0; i < 5; ++i)
+          t[i] = fmax3(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
+        t[5] = __uint_as_float(v[15]);
+        bmax[blk] = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]));
       }
       const float hmax = fmaxf(fmaxf(bmax[0], bmax[1]), fmaxf(bmax[2], bmax[3]));
       xmax[((j & 1) * 2 + h) * 128 + r] = hmax;
@@ -434,10 +433,15 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + 32, o1);
           tmem_ld_wait(o0);
           tmem_ld_wait(o1);
+          const float2 a2 = make_float2(a_pend, a_pend), s2 = make_float2(s1_pend, s1_pend);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            o_out[i] = fmaf(a_pend, o_out[i], s1_pend * __uint_as_float(o0[i]));
-            o_out[32 + i] = fmaf(a_pend, o_out[32 + i], s1_pend * __uint_as_float(o1[i]));
+          for (int i = 0; i < 32; i += 2) {
+            const float2 t0 = fmul2(s2, make_float2(__uint_as_float(o0[i]), __uint_as_float(o0[i + 1])));
+            const float2 t1 = fmul2(s2, make_float2(__uint_as_float(o1[i]), __uint_as_float(o1[i + 1])));
+            const float2 r0 = ffma2(a2, make_float2(o_out[i], o_out[i + 1]), t0);
+            const float2 r1 = ffma2(a2, make_float2(o_out[32 + i], o_out[32 + i + 1]), t1);
+            o_out[i] = r0.x; o_out[i + 1] = r0.y;
+            o_out[32 + i] = r1.x; o_out[32 + i + 1] = r1.y;
           }
         } else {
           uint32_t o[32];
