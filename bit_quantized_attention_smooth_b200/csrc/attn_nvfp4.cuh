@@ -13,17 +13,18 @@
 //   O_out  = alpha O_out + s1 O_in  (every tile: s1 changes per tile),  l = alpha l + rowsum(P~)
 //   O      = O_out / l
 //
-// CTA = one 128-row query tile of one (b, h); 10 warps:
-//   warps 0-3  softmax, left half: keys 0-63 of each key tile and output
-//              columns [0, D/2) of row 32 w + lane (TMEM lane quarter w)
-//   warps 4-7  softmax, right half: keys 64-127, output columns [D/2, D)
-//   warp 8     TMA producer (codes by tensor maps, scale factors by 1-D bulk copies)
-//   warp 9     TMEM allocator and single-thread MMA issuer; it also moves the
+// CTA = one 128-row query tile of one (b, h); 18 warps:
+//   warps 0-15 softmax: warp w serves row 32 (w mod 4) + lane (TMEM lane
+//              quarter w mod 4) and key quarter k = w / 4: keys 32 k .. 32 k + 31
+//              of each key tile (two 16-key scale blocks) and output columns
+//              [k D / 4, (k + 1) D / 4)
+//   warp 16    TMA producer (codes by tensor maps, scale factors by 1-D bulk copies)
+//   warp 17    TMEM allocator and single-thread MMA issuer; it also moves the
 //              scale factors from shared to tensor memory (tcgen05.cp 32x128b.warpx4)
-// The two threads of a row exchange their halves' maxima through shared
-// memory (a bounded two-warp mbarrier per lane quarter); each quantises its
-// 64 keys of P (exactly the 64-key slice of one block-scaled MMA) and keeps
-// its half of the outer accumulator in registers.
+// The four threads of a row exchange their quarters' maxima through shared
+// memory (a bounded four-warp mbarrier per lane quarter); each quantises its
+// 32 keys of P and keeps its quarter of the outer accumulator in registers.
+// Four softmax warps per SM sub-partition hide each other's latency.
 // TMEM columns: S [0,128) [128,256), O_in [256,256+D), scale factors from 384.
 // Scale factors of a 128-row operand and a 64-value slice of the contraction
 // axis occupy 4 columns: row m at lane m % 32 of every sub-partition, column
@@ -39,7 +40,8 @@
 
 namespace sattn {
 
-constexpr int kF4Threads = 320;
+constexpr int kF4Threads = 576;
+constexpr int kF4SoftmaxWarps = 16;
 constexpr float kLog2_2688 = 11.392317422778761f;   // log2(448 * 6)
 constexpr float kLog2_6 = 2.584962500721156f;       // log2(6)
 
@@ -71,10 +73,10 @@ struct AttnF4Smem {
   static constexpr int kSfK = kSfQ + kSfQK;
   static constexpr int kSfVo = kSfK + kKVStages * kSfQK;
   static constexpr int kSfPo = kSfVo + kKVStages * kSfV;
-  static constexpr int kX = kSfPo + 2 * kSfP;          // float [2 phases][2 halves][128] + [2][128]
-  static constexpr int kBar = kX + (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr int kX = kSfPo + 2 * kSfP;          // float [2 phases][4 quarters][128] + [4][128]
+  static constexpr int kBar = kX + (2 * 4 * 128 + 4 * 128) * 4;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
-  // p_full[2], pv_done[2], pair[4], drain
+  // p_full[2], pv_done[2], quad[4], drain
   static constexpr int kNumBars = 1 + 4 * kKVStages + 8 + 4 + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 256;     // 256 bytes of slack after the last buffer
@@ -159,10 +161,10 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   uint64_t *s_free = s_full + 2;            // [2]
   uint64_t *p_full = s_free + 2;            // [2]
   uint64_t *pv_done = p_full + 2;           // [2]
-  uint64_t *pair = pv_done + 2;             // [lane quarter]
-  uint64_t *drain_bar = pair + 4;
-  float *xmax = reinterpret_cast<float *>(smem + L::kX);                  // [2][2][128]
-  float *xl = reinterpret_cast<float *>(smem + L::kX + 2 * 2 * 128 * 4);  // [2][128]
+  uint64_t *quad = pv_done + 2;             // [lane quarter]: the four key quarters of the rows
+  uint64_t *drain_bar = quad + 4;
+  float *xmax = reinterpret_cast<float *>(smem + L::kX);                  // [2][4][128]
+  float *xl = reinterpret_cast<float *>(smem + L::kX + 2 * 4 * 128 * 4);  // [4][128]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
@@ -176,11 +178,11 @@ __global__ void __launch_bounds__(kF4Threads, 1)
                         : static_cast<int>(blockIdx.x);
   const int nkv = CAUSAL ? min(qt + 1, nkv_all) : nkv_all;
 
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (tid == 256) {
+  if (tid == 512) {
     mbar_init(q_full, 1);
     for (int s = 0; s < kKVStages; ++s) {
       mbar_init(&k_full[s], 1);
@@ -190,16 +192,16 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 8);   // one arrival per softmax warp
-      mbar_init(&p_full[b], 8);
+      mbar_init(&s_free[b], kF4SoftmaxWarps);   // one arrival per softmax warp
+      mbar_init(&p_full[b], kF4SoftmaxWarps);
       mbar_init(&pv_done[b], 1);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&pair[i], 2);
+    for (int i = 0; i < 4; ++i) mbar_init(&quad[i], 4);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (tid == 288) {
+  if (tid == 544) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       int last_j = -1;
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdQK = idesc_nvfp4(kTile, kTile);
@@ -311,60 +313,66 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax warps
-    constexpr int kHalfD = D / 2;
-    const int h = warp >> 2;                          // half of the row
+    constexpr int kQD = D / 4;                        // output columns per warp
+    const int kq = warp >> 2;                         // key quarter of the row
     const int wq = warp & 3;                          // TMEM lane quarter
     const int r = wq * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const int row_g = qt * kTile + r;
     const float cl = args.sm_log2;                    // S is already dequantised by the MMA
-    float o_out[kHalfD];
+    float o_out[kQD];
 #pragma unroll
-    for (int i = 0; i < kHalfD; ++i) o_out[i] = 0.f;
-    float m_ref = -INFINITY, l = 0.f;                 // l: this half's share of the row sum
+    for (int i = 0; i < kQD; ++i) o_out[i] = 0.f;
+    float m_ref = -INFINITY, l = 0.f;                 // l: this quarter's share of the row sum
     float a_pend = 0.f, s1_pend = 0.f;                // factors of the tile whose P V is pending
     bool ok = true;
+    // this warp's output columns of O_in, read as one or two 16-column loads
+    auto load_oin = [&](uint32_t (&o)[kQD]) {
+      const uint32_t base = tmem + lane_base + kOin + kq * kQD;
+      if constexpr (kQD == 32) {
+        tmem_ld_32x32b_x32(base, o);
+        tmem_ld_wait(o);
+      } else {
+        tmem_ld_32x32b_x16(base, o);
+        tmem_ld_wait(o);
+      }
+    };
 
     for (int j = 0; j < nkv && ok; ++j) {
       const int b = j & 1;
       if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t s_tmem = tmem + lane_base + b * kTile + h * 64;
-      uint32_t sa[32], sb[32];
-      tmem_ld_32x32b_x32(s_tmem, sa);
-      tmem_ld_32x32b_x32(s_tmem + 32, sb);
+      uint32_t sa[32];
+      tmem_ld_32x32b_x32(tmem + lane_base + b * kTile + kq * 32, sa);
       tmem_ld_wait(sa);
-      tmem_ld_wait(sb);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[b]);          // S_b may take Q K_{j+2}^T
       const bool masked = ((j == nkv_all - 1) && (N & (kTile - 1))) || (CAUSAL && j == qt);
       if (masked) {
-        const int kv0 = j * kTile + h * 64;
+        const int kv0 = j * kTile + kq * 32;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < 32; ++i)
           if (kv0 + i >= N || (CAUSAL && kv0 + i > row_g)) sa[i] = __float_as_uint(-INFINITY);
-          if (kv0 + 32 + i >= N || (CAUSAL && kv0 + 32 + i > row_g)) sb[i] = __float_as_uint(-INFINITY);
-        }
       }
-      // maxima of the four 16-key blocks of this half, then the row max via the partner
-      float bmax[4];
+      // maxima of the two 16-key blocks of this quarter, then the row max via the other quarters
+      float bmax[2];
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
-        const uint32_t *v = (blk < 2 ? sa : sb) + (blk & 1) * 16;
+      for (int hb = 0; hb < 2; ++hb) {
+        const uint32_t *v = sa + hb * 16;
         float t[6];
 #pragma unroll
         for (int i = 0; i < 5; ++i)
           t[i] = fmax3(__uint_as_float(v[3 * i]), __uint_as_float(v[3 * i + 1]), __uint_as_float(v[3 * i + 2]));
         t[5] = __uint_as_float(v[15]);
-        bmax[blk] = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]));
+        bmax[hb] = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]));
       }
-      const float hmax = fmaxf(fmaxf(bmax[0], bmax[1]), fmaxf(bmax[2], bmax[3]));
-      xmax[((j & 1) * 2 + h) * 128 + r] = hmax;
+      float *xm = xmax + (j & 1) * 4 * 128;
+      xm[kq * 128 + r] = fmaxf(bmax[0], bmax[1]);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pair[wq]);
-      if (!mbar_wait(&pair[wq], j & 1, abort_flag)) { ok = false; break; }
-      const float tmax = fmaxf(hmax, xmax[((j & 1) * 2 + (1 - h)) * 128 + r]);
+      if (lane == 0) mbar_arrive(&quad[wq]);
+      if (!mbar_wait(&quad[wq], j & 1, abort_flag)) { ok = false; break; }
+      const float tmax = fmaxf(fmax3(xm[r], xm[128 + r], xm[256 + r]), xm[384 + r]);
       const float m_tile = tmax * cl;                   // finite: every processed tile has a valid key
       const float m_new = fmaxf(m_ref, m_tile);
       const float alpha = ex2_approx(m_ref - m_new);
@@ -372,83 +380,64 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       const float moff = m_tile - kLog2_2688;           // P2 = 2^(S2 - moff) <= 2688
       const float moff6 = moff + kLog2_6;
 
-      // two-stage NVFP4 quantisation of this half of P into buffer b (key slice h)
+      // two-stage NVFP4 quantisation of this quarter of P into buffer b
       if (!mbar_wait(&pv_done[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       uint8_t *prow = smem + L::kP + b * L::kPBytes + r * 64;
-      uint8_t *psf = smem + L::kSfPo + b * L::kSfP + h * 512;
+      uint8_t *psf = smem + L::kSfPo + b * L::kSfP + (kq >> 1) * 512;   // 64-key slice of the quarter
       float psum = 0.f;
       const float2 cl2 = make_float2(cl, cl);
+      uint32_t w[4];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t w[4];
+      for (int hb = 0; hb < 2; ++hb) {
+        const int blk = (kq & 1) * 2 + hb;                // 16-key block within the 64-key slice
+        // scale = E4M3(block max of P2 / 6): the division by 6 folds into the exponent
+        const float amax6 = ex2_approx(fmaf(bmax[hb], cl, -moff6));
+        const uint32_t sc_code = cvt_e4m3x2(amax6, 0.f) & 0xFFu;
+        const float sc = e4m3_to_float(sc_code);
+        psf[sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
+        // P2 / scale = 2^(S2 - moff - log2 scale): the division folds into the
+        // exponent's constant; the block's P2 sum is scale * sum(P2 / scale).
+        const bool live = sc > 0.f;
+        const float lsc = live ? __log2f(sc) : 0.f;
+        const float2 nb2 = make_float2(-(moff + lsc), -(moff + lsc));
+        float2 bsum = make_float2(0.f, 0.f);
+        uint32_t bytes[8];
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int blk = 2 * q + hb;                     // 16-key block within this half
-          // scale = E4M3(block max of P2 / 6): the division by 6 folds into the exponent
-          const float amax6 = ex2_approx(fmaf(bmax[blk], cl, -moff6));
-          const uint32_t sc_code = cvt_e4m3x2(amax6, 0.f) & 0xFFu;
-          const float sc = e4m3_to_float(sc_code);
-          psf[sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
-          // P2 / scale = 2^(S2 - moff - log2 scale): the division folds into the
-          // exponent's constant; the block's P2 sum is scale * sum(P2 / scale).
-          const bool live = sc > 0.f;
-          const float lsc = live ? __log2f(sc) : 0.f;
-          const float2 nb2 = make_float2(-(moff + lsc), -(moff + lsc));
-          float2 bsum = make_float2(0.f, 0.f);
-          uint32_t bytes[8];
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const uint32_t v0 = q == 0 ? sa[hb * 16 + i] : sb[hb * 16 + i];
-            const uint32_t v1 = q == 0 ? sa[hb * 16 + i + 1] : sb[hb * 16 + i + 1];
-            const float2 x = ffma2(make_float2(__uint_as_float(v0), __uint_as_float(v1)), cl2, nb2);
-            const float2 y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            bsum = fadd2(bsum, y);
-            bytes[i >> 1] = cvt_e2m1x2(y.x, y.y);
-          }
-          if (live) psum = fmaf(sc, bsum.x + bsum.y, psum);
-          else {
-            // a block whose scale rounds to 0 has all-zero codes; its P2 values
-            // (below 6 * 2^-10 of 2688) still count towards the row sum
-#pragma unroll
-            for (int i = 0; i < 8; ++i) bytes[i] = 0u;
-            psum += (bsum.x + bsum.y);
-          }
-          w[2 * hb] = __byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040), __byte_perm(bytes[2], bytes[3], 0x0040), 0x5410);
-          w[2 * hb + 1] = __byte_perm(__byte_perm(bytes[4], bytes[5], 0x0040), __byte_perm(bytes[6], bytes[7], 0x0040), 0x5410);
+        for (int i = 0; i < 16; i += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(sa[hb * 16 + i]), __uint_as_float(sa[hb * 16 + i + 1])),
+                                 cl2, nb2);
+          const float2 y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          bsum = fadd2(bsum, y);
+          bytes[i >> 1] = cvt_e2m1x2(y.x, y.y);
         }
-        // 16 bytes = keys h*64 + q*32 .. +31; 64-byte swizzled K-major row
-        const int c16 = h * 2 + q;
-        *reinterpret_cast<uint4 *>(prow + ((c16 ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (live) psum = fmaf(sc, bsum.x + bsum.y, psum);
+        else {
+          // a block whose scale rounds to 0 has all-zero codes; its P2 values
+          // (below 6 * 2^-10 of 2688) still count towards the row sum
+#pragma unroll
+          for (int i = 0; i < 8; ++i) bytes[i] = 0u;
+          psum += (bsum.x + bsum.y);
+        }
+        w[2 * hb] = __byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040), __byte_perm(bytes[2], bytes[3], 0x0040), 0x5410);
+        w[2 * hb + 1] = __byte_perm(__byte_perm(bytes[4], bytes[5], 0x0040), __byte_perm(bytes[6], bytes[7], 0x0040), 0x5410);
       }
+      // 16 bytes = keys 32 kq .. 32 kq + 31; 64-byte swizzled K-major row
+      *reinterpret_cast<uint4 *>(prow + ((kq ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
 
-      // flush the previous tile: O_out = a O_out + s1 O_in (this half of the columns)
+      // flush the previous tile: O_out = a O_out + s1 O_in (this quarter of the columns)
       if (j > 0) {
         const int t = j - 1;
         if (!mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if constexpr (kHalfD == 64) {
-          // both 32-column chunks behind one wait
-          uint32_t o0[32], o1[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD, o0);
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + 32, o1);
-          tmem_ld_wait(o0);
-          tmem_ld_wait(o1);
-          const float2 a2 = make_float2(a_pend, a_pend), s2 = make_float2(s1_pend, s1_pend);
+        uint32_t o[kQD];
+        load_oin(o);
+        const float2 a2 = make_float2(a_pend, a_pend), s2 = make_float2(s1_pend, s1_pend);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 t0 = fmul2(s2, make_float2(__uint_as_float(o0[i]), __uint_as_float(o0[i + 1])));
-            const float2 t1 = fmul2(s2, make_float2(__uint_as_float(o1[i]), __uint_as_float(o1[i + 1])));
-            const float2 r0 = ffma2(a2, make_float2(o_out[i], o_out[i + 1]), t0);
-            const float2 r1 = ffma2(a2, make_float2(o_out[32 + i], o_out[32 + i + 1]), t1);
-            o_out[i] = r0.x; o_out[i + 1] = r0.y;
-            o_out[32 + i] = r1.x; o_out[32 + i + 1] = r1.y;
-          }
-        } else {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD, o);
-          tmem_ld_wait(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o_out[i] = fmaf(a_pend, o_out[i], s1_pend * __uint_as_float(o[i]));
+        for (int i = 0; i < kQD; i += 2) {
+          const float2 tt = fmul2(s2, make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])));
+          const float2 rr = ffma2(a2, make_float2(o_out[i], o_out[i + 1]), tt);
+          o_out[i] = rr.x;
+          o_out[i + 1] = rr.y;
         }
       }
       l = fmaf(alpha, l, s1 * psum);
@@ -463,32 +452,28 @@ __global__ void __launch_bounds__(kF4Threads, 1)
 
     // ---------------------------------------------------------- epilogue
     if (ok && nkv > 0) {
-      xl[h * 128 + r] = l;
+      xl[kq * 128 + r] = l;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pair[wq]);
+      if (lane == 0) mbar_arrive(&quad[wq]);
       const int t = nkv - 1;
-      if (mbar_wait(&pair[wq], nkv & 1, abort_flag) && mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) {
+      if (mbar_wait(&quad[wq], nkv & 1, abort_flag) && mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) {
         tc_fence_after();
-        const float inv_l = 1.f / (xl[r] + xl[128 + r]);
-        OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D + h * kHalfD;
+        const float inv_l = 1.f / ((xl[r] + xl[128 + r]) + (xl[256 + r] + xl[384 + r]));
+        OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D + kq * kQD;
+        uint32_t o[kQD];
+        load_oin(o);
+        uint32_t packed[kQD / 2];
 #pragma unroll
-        for (int ch = 0; ch < kHalfD / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOin + h * kHalfD + ch * 32, o);
-          tmem_ld_wait(o);
-          uint32_t packed[16];
+        for (int i = 0; i < kQD; i += 2) {
+          const float o0 = fmaf(a_pend, o_out[i], s1_pend * __uint_as_float(o[i])) * inv_l;
+          const float o1 = fmaf(a_pend, o_out[i + 1], s1_pend * __uint_as_float(o[i + 1])) * inv_l;
+          packed[i >> 1] = pack2_out<OutT>(o0, o1);
+        }
+        if (row_g < N) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float o0 = fmaf(a_pend, o_out[ch * 32 + i], s1_pend * __uint_as_float(o[i])) * inv_l;
-            const float o1 = fmaf(a_pend, o_out[ch * 32 + i + 1], s1_pend * __uint_as_float(o[i + 1])) * inv_l;
-            packed[i >> 1] = pack2_out<OutT>(o0, o1);
-          }
-          if (row_g < N) {
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + ch * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
-          }
+          for (int u = 0; u < kQD / 8; ++u)
+            dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
         }
       }
     }
@@ -496,7 +481,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
