@@ -369,7 +369,7 @@ HostPipe g_host[kMaxDevices];
 
 // Chunks per call: enough to overlap the copies with the compute, few enough
 // that each chunk still fills the GPU.
-constexpr int kHostChunks = 4;
+constexpr int kHostChunks = 12;
 constexpr size_t kHostSlotCap = size_t(1) << 30;   // device bytes of one slot at most
 
 bool host_pipe_init(HostPipe &p) {

@@ -101,7 +101,7 @@ int sattn_fwd(const void *q, const void *k, const void *v, void *out,
 /* sattn_fwd on HOST buffers: q, k, v and out are host pointers ([B, H, N, d],
  * same element type and layout as sattn_fwd); pinned (page-locked) memory lets
  * the copies run asynchronously, pageable memory works but serializes them.
- * The call splits the B*H heads into a few chunks and pipelines them: chunk c
+ * The call splits the B*H heads into up to 12 chunks and pipelines them: chunk c
  * is copied to the device on one stream, quantized and attended on one of two
  * compute streams, and copied back on a fourth stream, so that the PCIe
  * transfers of one chunk overlap the compute of the others.  Attention heads
