@@ -367,8 +367,9 @@ struct HostPipe {
 std::mutex g_host_mutex;
 HostPipe g_host[kMaxDevices];
 
-// Chunks per call: enough to overlap the copies with the compute, few enough
-// that each chunk still fills the GPU.
+// Chunks per call: enough that the first copy in and the last copy out (the
+// pipeline's fill and drain) are short; a chunk smaller than the GPU is fine,
+// since the two compute streams let neighbouring chunks share the SMs.
 constexpr int kHostChunks = 12;
 constexpr size_t kHostSlotCap = size_t(1) << 30;   // device bytes of one slot at most
 
