@@ -15,8 +15,9 @@
 // overwrites O_in.  When a row's running max grows, O_out is rescaled by
 // alpha = 2^(m_old - m_new) through a per-row factor (O_out = beta * o_out,
 // beta *= alpha), and inside a group that row's O_in in TMEM is multiplied by
-// alpha (per warp, only when some lane of the warp needs it).  Both happen after P of the tile has
-// been written, when the previous P V has long completed.  Finally
+// alpha (per warp, only when some lane of the warp needs it).  Both happen
+// after P of the tile has been written, when the previous P V has long
+// completed.  Finally
 //   O = (O_out + O_in) * s_v[c] / (448 l).
 //
 // CTA = two 128-row query tiles (A, B) of one (b, h) sharing every K/V tile;
@@ -29,8 +30,10 @@
 //              the softmax warpgroups through setmaxnreg)
 // Two softmax warps per SM sub-partition hide each other's latency.  TMEM
 // columns: S_A [0,128), S_B [128,256), O_in_A [256,256+D), O_in_B
-// [256+D, 256+2D).  Each softmax warp reads its S twice (row max, then P), so
-// that the 128 outer-accumulator registers and one 32-column chunk fit.
+// [256+D, 256+2D).  Each softmax warp reads its S twice (row max, then P),
+// 64 columns at a time (two 32-column loads behind one wait), so that the 128
+// outer-accumulator registers and the 64 score registers fit in the softmax
+// warps' 232.
 #pragma once
 
 #include <cuda_bf16.h>
