@@ -1,8 +1,8 @@
 /*
  * sattn -- SageAttention-style quantized attention forward for NVIDIA B200 (sm_100a).
  *
- * C ABI of libsattn.so.  All entry points are plain C: device pointers, sizes,
- * a CUDA stream.  No entry point throws or aborts; each returns a status code
+ * C ABI of libsattn.so.  All entry points are plain C: device pointers (host
+ * pointers for sattn_fwd_host), sizes, a CUDA stream.  No entry point throws or aborts; each returns a status code
  * (sattn_status_t) and never synchronizes the stream unless stated.
  *
  * The operation (TurboDiffusion explainer, wxsanhe.com post 64219, section 1
@@ -28,7 +28,8 @@
  *
  * Tensor layout (all modes): q, k, v, out are contiguous [B, H, N, d] ("BHND"),
  * element type bf16 (default) or fp16 (mode | SATTN_FP16_IO); out has the
- * input's element type.  Pointers must be 16-byte aligned device pointers.
+ * input's element type.  Device pointers must be 16-byte aligned (the host
+ * pointers of sattn_fwd_host may have any alignment).
  * Supported: d in {64, 128}; N >= 1; B*H >= 1; B*H*N*d < 2^31.
  * sm_scale <= 0 selects 1/sqrt(d).  causal masks key j > query i.
  *
