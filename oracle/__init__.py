@@ -10,8 +10,10 @@ What it computes
 * ``attention.attn_exact`` -- the plain definition O = softmax(Q K^T * s) V in
   float64 (optionally causal).  Target of the cosine criterion.
 * ``attention.attn_quant_emul_i8f8`` -- the INT8-QK / FP8-PV scheme step by step:
-  K smoothed by its per-channel token mean, per-block INT8 Q and K, per-channel
-  FP8 V, FP8 P with a static 448 scale, online softmax over 128-key tiles.
+  K smoothed by its per-channel token mean, per-block (or per-token) INT8 Q and
+  per-block INT8 K, per-channel FP8 V, FP8 P with a static scale, online
+  softmax over 128-key tiles whose reference max moves exactly (tau = 0) or
+  lazily (only when a tile's max is more than tau above it).
   Quantiser arithmetic is float32 exactly as the device performs it; everything
   after the codes is float64.
 * ``attention.attn_quant_emul_nvfp4`` -- the NVFP4 microscaled scheme with the

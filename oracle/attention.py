@@ -11,10 +11,15 @@ The emulations follow the order of the method:
 
 1. quantise (``quant.quantize_head_*``);
 2. for each query row, sweep the keys in tiles of ``block_kv`` with an online
-   softmax: running max m, P~ = 2^(S - m) relative to the running max after the
-   tile, rescale factor alpha = 2^(m_old - m_new), l accumulated from the
-   unquantised P~ (FlashAttention-style streaming, which the TurboDiffusion
-   explainer, wxsanhe.com post 64219, section 1, says the method replaces);
+   softmax: reference max m, P~ = 2^(S - m), rescale factor
+   alpha = 2^(m_old - m_new), l accumulated from the unquantised P~
+   (FlashAttention-style streaming, which the TurboDiffusion explainer,
+   wxsanhe.com post 64219, section 1, says the method replaces).  The pages do
+   not say when the reference max moves.  ``tau`` = 0 is the exact running max
+   (m is the row max of every key seen so far, so P~ <= 1); ``tau`` > 0 is the
+   lazy policy: m moves to a tile's row max only when that max exceeds m by
+   more than ``tau``, so that P~ <= 2^tau and the accumulators are rescaled
+   only when the max has grown by more than that;
 3. quantise P~ per tile and accumulate its product with the quantised V.
 
 Scores are carried in the base-2 domain: S2 = S * sm_scale * log2(e).
@@ -76,13 +81,15 @@ def attn_exact(q, k, v, causal=False, sm_scale=None, heads=None, rows=None):
     return out
 
 
-def _online_softmax(S2, valid, tile, p_quant, pv):
+def _online_softmax(S2, valid, tile, p_quant, pv, tau=0.0):
     """Generic streaming softmax over key tiles.
 
     S2: [R, N] float64 base-2 scores; valid: [R, N] bool.
     p_quant(P~ tile) -> (Pq tile, row factor) : quantised P and the factor that
         multiplies the tile's contribution (1 for static scales).
     pv(Pq, j0, j1) -> [R, d] product of the quantised P tile with V rows j0:j1.
+    tau: the reference max of a row moves to the tile's row max only when that
+        max exceeds it by more than tau (0: exact running max).
     Returns (acc [R, d], l [R]) with O = acc / l up to the V scale.
     """
     R, N = S2.shape
@@ -92,7 +99,8 @@ def _online_softmax(S2, valid, tile, p_quant, pv):
     for j0 in range(0, N, tile):
         j1 = min(j0 + tile, N)
         St = np.where(valid[:, j0:j1], S2[:, j0:j1], -np.inf)
-        m_new = np.maximum(m, St.max(axis=1))
+        m_tile = St.max(axis=1)
+        m_new = np.where(m_tile > m + tau, m_tile, m)
         m_use = np.where(np.isneginf(m_new), 0.0, m_new)
         P = np.exp2(St - m_use[:, None])                 # 0 where masked
         alpha = np.exp2(np.where(np.isneginf(m), -np.inf, m - m_use))
@@ -105,10 +113,11 @@ def _online_softmax(S2, valid, tile, p_quant, pv):
 
 
 def attn_online_unquantised(q, k, v, causal=False, sm_scale=None, heads=None,
-                            rows=None, block_kv=128):
+                            rows=None, block_kv=128, tau=0.0):
     """The same tiled online softmax with every quantiser replaced by identity.
 
-    Equal to ``attn_exact`` up to float64 rounding; pins the streaming logic.
+    Equal to ``attn_exact`` up to float64 rounding for any ``tau`` (the
+    reference max cancels in acc / l); pins the streaming logic.
     """
     B, H, N, d = q.shape
     s = default_scale(d, sm_scale)
@@ -121,7 +130,7 @@ def attn_online_unquantised(q, k, v, causal=False, sm_scale=None, heads=None,
         acc, l = _online_softmax(
             S2, _valid_mask(rows, cols, N, causal), block_kv,
             lambda P: (P, np.ones(P.shape[0])),
-            lambda Pq, j0, j1: Pq @ vh[j0:j1])
+            lambda Pq, j0, j1: Pq @ vh[j0:j1], tau)
         out[t] = acc / l[:, None]
     return out
 
@@ -137,16 +146,22 @@ def int8_scores(qh, kh):
 
 
 def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
-                         block_q=128, block_kv=128):
+                         block_q=128, block_kv=128, tau=0.0):
     """INT8 QK^T / FP8 PV emulation (the I8QK_F8PV mode).
 
     Steps (TurboDiffusion explainer, section 1: QK in INT8, PV in FP8, outlier
     smoothing, two-level accumulation; tag page SageAttention3 summary [17]:
     per-block INT8 for Q/K):
       S2[i,j] = (q8_i . k8_j) * s_q[blk(i)] * s_k[blk(j)] * sm_scale * log2 e
-      P~ tile = 2^(S2 - m_running);  p8 = E4M3(448 * P~)
+      P~ tile = 2^(S2 - m);  p8 = E4M3(c_P * P~),  c_P = 448 * 2^-tau
       acc     = alpha * acc + p8 @ v8;  l = alpha * l + rowsum(P~)
-      O       = acc * s_v[c] / (448 * l)
+      O       = acc * s_v[c] / (c_P * l)
+    m is the reference max of the row (see ``tau`` in the module docstring):
+    P~ <= 2^tau, so the static scale c_P maps the largest possible P~ onto
+    E4M3's largest finite value, 448.  ``block_q`` = 1 gives one Q scale per
+    token, the finest token granularity ("thread-level quantization", QbitAI
+    reprint, txrjy.com, SageAttention paragraph, with one query row per
+    softmax thread).
     """
     B, H, N, d = q.shape
     s = default_scale(d, sm_scale)
@@ -160,11 +175,12 @@ def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=
         sq_rows = z["sq"][rows // block_q].astype(np.float64)
         sk_cols = z["sk"][cols // block_kv].astype(np.float64)
         S2 = Sint * sq_rows[:, None] * sk_cols[None, :] * (s * LOG2E)
+        c_p = P_SCALE_FP8 * 2.0 ** -tau
         acc, l = _online_softmax(
             S2, _valid_mask(rows, cols, N, causal), block_kv,
-            lambda P: (e4m3_round(P_SCALE_FP8 * P), np.ones(P.shape[0])),
-            lambda Pq, j0, j1: Pq @ v8[j0:j1])
-        out[t] = acc * z["sv"].astype(np.float64)[None, :] / (P_SCALE_FP8 * l[:, None])
+            lambda P: (e4m3_round(c_p * P), np.ones(P.shape[0])),
+            lambda Pq, j0, j1: Pq @ v8[j0:j1], tau)
+        out[t] = acc * z["sv"].astype(np.float64)[None, :] / (c_p * l[:, None])
     return out
 
 

@@ -52,13 +52,18 @@ def _i8(x, s):
     return max(-127, min(127, r))
 
 
-def i8f8_head(Q, K, V, causal, sm_scale, blk=128):
-    """One head, lists of float32 rows.  Returns list of output rows (floats)."""
+def i8f8_head(Q, K, V, causal, sm_scale, blk=128, blk_q=None, tau=0.0):
+    """One head, lists of float32 rows.  Returns list of output rows (floats).
+
+    blk: token block of the K scales and the key tile; blk_q: token block of
+    the Q scales (default blk); tau: the row's reference max moves to a tile's
+    max only when that max is more than tau above it."""
     N, d = len(Q), len(Q[0])
+    blk_q = blk if blk_q is None else blk_q
     mu = _kmean(K, N, d)
     Kp = [[F32(F32(K[n][c]) - mu[c]) for c in range(d)] for n in range(N)]
 
-    def block_q8(X):
+    def block_q8(X, blk):
         codes, scales = [], []
         for b0 in range(0, N, blk):
             amax = F32(0.0)
@@ -71,8 +76,8 @@ def i8f8_head(Q, K, V, causal, sm_scale, blk=128):
                 codes.append([_i8(X[n][c], s) for c in range(d)])
         return codes, scales
 
-    q8, sq = block_q8(Q)
-    k8, sk = block_q8(Kp)
+    q8, sq = block_q8(Q, blk_q)
+    k8, sk = block_q8(Kp, blk)
     sv = []
     for c in range(d):
         amax = F32(0.0)
@@ -82,6 +87,7 @@ def i8f8_head(Q, K, V, causal, sm_scale, blk=128):
     v8 = [[fp8(F32(F32(V[n][c]) / sv[c])) for c in range(d)] for n in range(N)]
 
     c2 = sm_scale / math.log(2.0)
+    cp = 448.0 / 2.0 ** tau             # static FP8 scale of P: 2^tau -> 448
     out = []
     for i in range(N):
         m, l = -math.inf, 0.0
@@ -93,21 +99,23 @@ def i8f8_head(Q, K, V, causal, sm_scale, blk=128):
                 if causal and j > i:
                     continue
                 dot = sum(q8[i][c] * k8[j][c] for c in range(d))
-                s2[j] = dot * float(sq[i // blk]) * float(sk[j // blk]) * c2
+                s2[j] = dot * float(sq[i // blk_q]) * float(sk[j // blk]) * c2
             if not s2:
                 continue
-            m_new = max(m, max(s2.values()))
+            top = max(s2.values())
+            m_new = top if (m == -math.inf or top - m > tau) else m
             alpha = 0.0 if m == -math.inf else 2.0 ** (m - m_new)
             l *= alpha
             acc = [a * alpha for a in acc]
             for j, sv2 in s2.items():
                 p = 2.0 ** (sv2 - m_new)
+                assert p <= 2.0 ** tau
                 l += p
-                p8 = fp8(448.0 * p)
+                p8 = fp8(cp * p)
                 for c in range(d):
                     acc[c] += p8 * v8[j][c]
             m = m_new
-        out.append([acc[c] * float(sv[c]) / (448.0 * l) for c in range(d)])
+        out.append([acc[c] * float(sv[c]) / (cp * l) for c in range(d)])
     return out
 
 

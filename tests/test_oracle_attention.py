@@ -74,6 +74,36 @@ def test_online_unquantised_equals_exact(N, causal):
     assert np.abs(a - c).max() < 1e-12
 
 
+@pytest.mark.parametrize("tau", [0.5, 4.0, 8.0])
+@pytest.mark.parametrize("N,causal", [(300, False), (300, True), (129, True)])
+def test_online_unquantised_lazy_max_equals_exact(N, causal, tau):
+    """The reference max cancels between acc and l: any lazy threshold gives exact attention."""
+    q, k, v, _ = _inputs(1, 2, N, 16, seed=N + 7)
+    q *= 3.0                                           # wide scores: the max moves often
+    a = A.attn_exact(q, k, v, causal=causal)
+    b = A.attn_online_unquantised(q, k, v, causal=causal, block_kv=16, tau=tau)
+    assert np.abs(a - b).max() < 1e-12
+
+
+@pytest.mark.parametrize("tau", [0.0, 2.0, 4.0])
+def test_lazy_max_bounds_p_and_moves_less_often(tau):
+    """P~ <= 2^tau in every tile; a larger tau moves the reference max no more often."""
+    rng = np.random.default_rng(3)
+    S2 = rng.standard_normal((64, 1024)) * 4.0
+    valid = np.ones_like(S2, dtype=bool)
+    seen = []
+
+    def pq(P):
+        seen.append(P.max())
+        return P, np.ones(P.shape[0])
+
+    acc, l = A._online_softmax(S2, valid, 64, pq, lambda P, j0, j1: P.sum(axis=1, keepdims=True), tau)
+    assert max(seen) <= 2.0 ** tau * (1 + 1e-15)
+    assert max(seen) > 2.0 ** tau * 0.5 or tau == 0.0  # the bound is approached
+    # sum_j P~_j / l == 1 whatever the reference
+    assert np.abs(acc[:, 0] / l - 1.0).max() < 1e-12
+
+
 def test_sampling_rows_and_heads_matches_full():
     q, k, v, _ = _inputs(2, 3, 150, 32, seed=9)
     full = A.attn_quant_emul_i8f8(q, k, v)
@@ -90,6 +120,17 @@ def test_i8f8_uniform_queries_give_mean_of_dequantised_v():
     _, k, v, _ = _inputs(1, 1, 300, 32, seed=2)
     q = np.zeros_like(k)
     o = A.attn_quant_emul_i8f8(q, k, v)[0]
+    v8, sv = Qz.quant_v_fp8(v[0, 0])
+    want = (e4m3_decode(v8) * sv.astype(np.float64)[None, :]).mean(axis=0)
+    assert np.abs(o - want[None, :]).max() < 1e-12
+
+
+@pytest.mark.parametrize("tau", [2.0, 4.0, 8.0])
+def test_i8f8_lazy_uniform_queries_give_mean_of_dequantised_v(tau):
+    """Q = 0: every P~ = 1 <= 2^tau, p8 = E4M3(448 * 2^-tau) is exact -> O = mean_j(s_v * v8_j)."""
+    _, k, v, _ = _inputs(1, 1, 300, 32, seed=2)
+    q = np.zeros_like(k)
+    o = A.attn_quant_emul_i8f8(q, k, v, tau=tau)[0]
     v8, sv = Qz.quant_v_fp8(v[0, 0])
     want = (e4m3_decode(v8) * sv.astype(np.float64)[None, :]).mean(axis=0)
     assert np.abs(o - want[None, :]).max() < 1e-12
@@ -130,6 +171,18 @@ def test_int8_block_quant_bounds():
         c = codes[b * 128:(b + 1) * 128].astype(np.float64)
         assert np.abs(c).max() == 127
         assert np.abs(blk - s[b] * c).max() <= s[b] * (0.5 + 127 * 2.0 ** -23)
+
+
+def test_int8_per_token_quant_bounds():
+    """block 1: one scale per token, every row reaches code +-127 and the half-step bound."""
+    q, _, _, _ = _inputs(1, 1, 50, 64, seed=16, q_outlier_frac=0.02)
+    x = q[0, 0]
+    codes, s = Qz.quant_int8_blocks(x, 1)
+    assert s.shape == (50,)
+    c = codes.astype(np.float64)
+    assert np.all(np.abs(c).max(axis=1) == 127)
+    assert np.all(np.abs(x.astype(np.float64) - s[:, None] * c) <= s[:, None] * (0.5 + 127 * 2.0 ** -23))
+    np.testing.assert_array_equal(s, (np.abs(x).max(axis=1) / np.float32(127)).astype(np.float32))
 
 
 def test_k_mean_and_smoothing():
@@ -191,6 +244,18 @@ def test_i8f8_matches_scalar_restatement(N, d, causal, dtype):
     s = 1.0 / math.sqrt(d)
     o = A.attn_quant_emul_i8f8(q, k, v, causal=causal, block_q=16, block_kv=16)[0]
     ref = scalar_ref.i8f8_head(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, s, blk=16)
+    assert np.abs(o - np.array(ref)).max() < 1e-9
+
+
+@pytest.mark.parametrize("N,d,causal,blk_q,tau", [(40, 16, False, 16, 2.0), (33, 32, True, 1, 0.0),
+                                                  (45, 16, True, 1, 1.0), (48, 16, False, 16, 8.0)])
+def test_i8f8_lazy_and_per_token_match_scalar_restatement(N, d, causal, blk_q, tau):
+    q, k, v, _ = _inputs(1, 1, N, d, seed=N + 3, q_outlier_frac=0.05)
+    q *= 2.0                                            # wide scores: the lazy max moves now and then
+    s = 1.0 / math.sqrt(d)
+    o = A.attn_quant_emul_i8f8(q, k, v, causal=causal, block_q=blk_q, block_kv=16, tau=tau)[0]
+    ref = scalar_ref.i8f8_head(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, s, blk=16,
+                               blk_q=blk_q, tau=tau)
     assert np.abs(o - np.array(ref)).max() < 1e-9
 
 
