@@ -35,7 +35,7 @@ import math
 import numpy as np
 
 from .formats import e4m3_round, e4m3_decode, int8_quantize  # noqa: F401
-from .quant import quantize_head_i8f8, quantize_head_nvfp4, nvfp4_dequant_rows, nvfp4_quant_rows
+from .quant import quantize_head_i8f8, quantize_head_nvfp4, nvfp4_dequant_rows, nvfp4_quant_rows, fp4_rows
 
 LOG2E = 1.0 / math.log(2.0)
 P_SCALE_FP8 = 448.0           # static scale of P~ in [0, 1] onto E4M3's range
@@ -184,7 +184,7 @@ def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=
     return out
 
 
-def two_stage_p_nvfp4(P):
+def two_stage_p_nvfp4(P, fmt="nvfp4"):
     """Two-stage quantisation of one P~ tile [R, T] (T <= 128 keys).
 
     Stage 1 (per row of the tile): s1 = rowmax(P~) / (448 * 6), s1 = 1 for an
@@ -192,18 +192,18 @@ def two_stage_p_nvfp4(P):
     second-stage E4M3 scales use their whole range.  Stage 2: NVFP4 blocks of
     16 keys on P2.  (Tag page, SageAttention3 summary, FP4 bullets [15][16]:
     two-stage quantisation fixes the narrow range of P's scale factors.)
+    ``fmt`` = "mxfp4" swaps the second stage for MXFP4 (the ablation).
     Returns (dequantised P2 [R, T] float64, s1 [R] float64).
     """
     r = P.max(axis=1)
     s1 = np.where(r > 0, r / P_STAGE1_DIV, 1.0)
     P2 = (P / s1[:, None]).astype(np.float32)
     T = P.shape[1]
-    codes, _, sc = nvfp4_quant_rows(P2)
-    return nvfp4_dequant_rows(codes, sc)[:, :T], s1
+    return fp4_rows(P2, fmt)[:, :T], s1
 
 
 def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
-                          block_kv=128):
+                          block_kv=128, fmt="nvfp4"):
     """NVFP4 microscaled emulation (the NVFP4 mode).
 
       Q^, K'^ : NVFP4 along channels;  V^ : NVFP4 along tokens
@@ -211,6 +211,9 @@ def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows
       per key tile: P~ = 2^(S2 - m_running); (P2^, s1) = two_stage_p_nvfp4(P~)
       acc     = alpha * acc + s1 * (P2^ @ V^);  l = alpha * l + rowsum(P~)
       O       = acc / l
+    ``fmt`` = "mxfp4" runs the same scheme with every FP4 operand in MXFP4
+    (1 x 32 blocks, E8M0 scales): the ablation that the tag page's
+    SageAttention3 summary, FP4 bullet [15], reports NVFP4 winning.
     """
     B, H, N, d = q.shape
     s = default_scale(d, sm_scale)
@@ -218,14 +221,21 @@ def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows
     out = np.empty((len(heads), len(rows), d))
     cols = np.arange(N)
     for t, (b, h) in enumerate(heads):
-        z = quantize_head_nvfp4(q[b, h], k[b, h], v[b, h])
-        qv = nvfp4_dequant_rows(z["q"], z["q_sc"])[:, :d]
-        kv = nvfp4_dequant_rows(z["k"], z["k_sc"])[:, :d]
-        vv = nvfp4_dequant_rows(z["vt"], z["vt_sc"])[:, :N].T      # [N, d]
+        if fmt == "nvfp4":
+            z = quantize_head_nvfp4(q[b, h], k[b, h], v[b, h])
+            qv = nvfp4_dequant_rows(z["q"], z["q_sc"])[:, :d]
+            kv = nvfp4_dequant_rows(z["k"], z["k_sc"])[:, :d]
+            vv = nvfp4_dequant_rows(z["vt"], z["vt_sc"])[:, :N].T      # [N, d]
+        else:
+            from .quant import k_channel_mean, smooth_k
+            kp = smooth_k(k[b, h], k_channel_mean(k[b, h]))
+            qv = fp4_rows(q[b, h], fmt)[:, :d]
+            kv = fp4_rows(kp, fmt)[:, :d]
+            vv = fp4_rows(np.ascontiguousarray(v[b, h].T), fmt)[:, :N].T
         S2 = (qv[rows] @ kv.T) * (s * LOG2E)
         acc, l = _online_softmax(
             S2, _valid_mask(rows, cols, N, causal), block_kv,
-            two_stage_p_nvfp4,
+            lambda P: two_stage_p_nvfp4(P, fmt),
             lambda Pq, j0, j1: Pq @ vv[j0:j1])
         out[t] = acc / l[:, None]
     return out

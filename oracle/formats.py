@@ -13,7 +13,8 @@ Formats
   magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.  Used with one unsigned E4M3 scale
   per 16 consecutive values (NVFP4 microscaling), which the SageAttention tag
   page (reportify.cn), SageAttention3 summary, FP4 bullet [15] names as the
-  chosen format.
+  chosen format, and, for the ablation the same bullet compares it with, with
+  one E8M0 power-of-two scale per 32 values (MXFP4, OCP Microscaling).
 
 Rounding is round-to-nearest-even on the value, then saturation to the largest
 finite magnitude ("satfinite"), which is the rounding the tensor-core
@@ -172,15 +173,46 @@ def e2m1_encode_bruteforce(x):
 
 
 # ----------------------------------------------------------------------------
+# E8M0 (the shared scale of the OCP MX formats, used by the MXFP4 ablation)
+# ----------------------------------------------------------------------------
+# 8 exponent bits, no sign, no mantissa: code c is 2^(c - 127), c = 255 is NaN.
+
+def e8m0_decode(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    return np.where(c == 255, np.nan, np.exp2((c - 127).astype(np.float64)))
+
+
+def mx_scale_code(amax, emax_elem):
+    """E8M0 code of the MX shared scale 2^(floor(log2 amax) - emax_elem).
+
+    This is the OCP Microscaling rule: the block's largest magnitude lands in
+    the element format's top binade (for E2M1, emax_elem = 2: [4, 8) before
+    the elements saturate at 6).  amax = 0 gives the smallest code (the block
+    is all zeros either way); NaN gives the NaN code.
+    """
+    a = np.asarray(amax, dtype=np.float64)
+    nan = np.isnan(a)
+    safe = np.where((a > 0) & ~nan, a, 1.0)
+    _, E = np.frexp(safe)                     # safe = f * 2^E, f in [0.5, 1): floor(log2) = E - 1
+    code = np.clip(E.astype(np.int64) - 1 - emax_elem + 127, 0, 254)
+    code = np.where(a > 0, code, 0)
+    return np.where(nan, 255, code).astype(np.uint8)
+
+
+# ----------------------------------------------------------------------------
 # INT8 with a float32 scale
 # ----------------------------------------------------------------------------
 
 def int8_quantize(x32, s32):
     """q = RNE(x / s) with the division in float32, clamped to [-127, 127].
 
-    ``x32`` and ``s32`` are float32 arrays that broadcast together.
+    ``x32`` and ``s32`` are float32 arrays that broadcast together.  A NaN
+    quotient (a NaN input or a NaN scale) gives code 0; its scale carries the
+    NaN on to the scores.
     """
     x32 = np.asarray(x32, dtype=np.float32)
     s32 = np.asarray(s32, dtype=np.float32)
-    y = (x32 / s32).astype(np.float32)          # IEEE float32 division
+    with np.errstate(invalid="ignore"):
+        y = (x32 / s32).astype(np.float32)      # IEEE float32 division
+    y = np.where(np.isnan(y), np.float32(0), y)
     return np.clip(np.rint(y), -127, 127).astype(np.int8)

@@ -26,12 +26,16 @@ Readings of the pages (which give no formulas):
   (float32 division, then E4M3 rounding), codes = E2M1(x / scale) with the
   division in float32; a block whose scale rounds to zero gets all-zero codes.
   No per-tensor second-level scale.
+* NaN inputs (the pages say nothing): every maximum propagates NaN, so a NaN
+  makes the scale it feeds NaN -- the rows of its Q block (or token), the K
+  channel mean and with it every K scale of the head, or one V channel's
+  scale -- and the outputs that use that scale are NaN.
 """
 
 import numpy as np
 
 from .formats import (e4m3_encode, e4m3_decode, e2m1_encode, e2m1_decode,
-                      int8_quantize)
+                      e8m0_decode, int8_quantize, mx_scale_code)
 
 INT8_MAX = np.float32(127.0)
 FP8_MAX = np.float32(448.0)
@@ -98,6 +102,36 @@ def nvfp4_quant_rows(x32, block=16):
     codes = e2m1_encode(y)
     codes = np.where(sc[:, :, None] == 0, np.uint8(0), codes).astype(np.uint8)
     return codes.reshape(r, Lp), sc_codes, sc
+
+
+def mxfp4_quant_rows(x32, block=32):
+    """MXFP4 along the last axis (the ablation of the tag page's FP4 bullet
+    [15]): blocks of 32 values, scale = E8M0 2^(floor(log2 max|x|) - 2),
+    codes = E2M1(x / scale) RNE satfinite (the division by a power of two is
+    exact).  Returns (codes [R, Lp], scale codes [R, Lp/32], scales float64),
+    Lp = L rounded up to 32, padding treated as zeros."""
+    x32 = np.asarray(x32, dtype=np.float32)
+    r, L = x32.shape
+    Lp = (L + block - 1) // block * block
+    xp = np.zeros((r, Lp), dtype=np.float32)
+    xp[:, :L] = x32
+    xb = xp.reshape(r, Lp // block, block).astype(np.float64)
+    sc_codes = mx_scale_code(np.max(np.abs(xb), axis=2), 2)
+    sc = e8m0_decode(sc_codes)
+    codes = e2m1_encode(xb / sc[:, :, None])
+    return codes.reshape(r, Lp), sc_codes, sc
+
+
+def fp4_rows(x32, fmt):
+    """Quantise-dequantise rows in an FP4 microscaling format ("nvfp4" or
+    "mxfp4"); float64 [R, Lp]."""
+    if fmt == "nvfp4":
+        codes, _, sc = nvfp4_quant_rows(x32)
+        return nvfp4_dequant_rows(codes, sc)
+    if fmt == "mxfp4":
+        codes, _, sc = mxfp4_quant_rows(x32)
+        return nvfp4_dequant_rows(codes, sc, block=32)
+    raise ValueError(fmt)
 
 
 def nvfp4_dequant_rows(codes, scales, block=16):

@@ -288,7 +288,7 @@ def test_nvfp4_two_stage_p_beats_one_stage():
     two = A.attn_quant_emul_nvfp4(q, k, v, rows=rows)
     orig = A.two_stage_p_nvfp4
 
-    def one_stage(P):
+    def one_stage(P, fmt="nvfp4"):
         codes, _, sc = Qz.nvfp4_quant_rows(P.astype(np.float32))
         return Qz.nvfp4_dequant_rows(codes, sc)[:, :P.shape[1]], np.ones(P.shape[0])
 
