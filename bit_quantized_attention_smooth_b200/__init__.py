@@ -19,13 +19,18 @@ LIB_PATH = os.path.join(_PKG, "libsattn.so")
 
 MODES = {"i8f8": 0, "nvfp4": 1}
 FP16_IO = 0x100
+Q_PER_TOKEN = 0x200
+# Lazy reference-max threshold of the I8QK_F8PV kernel (SATTN_I8F8_LAZY_TAU in
+# include/sattn.h): the row max moves only when a key tile exceeds it by more
+# than this many powers of two, and P's static FP8 scale is 448 * 2^-tau.
+I8F8_LAZY_TAU = 4.0
 STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
           3: "SATTN_ERR_WORKSPACE", 4: "SATTN_ERR_CUDA"}
 
 # Every entry point declared in include/sattn.h.
 EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
            "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc",
-           "sattn_fwd_host")
+           "sattn_fwd_host", "sattn_kernel_launches", "sattn_debug_set_wait_limit")
 
 
 class SattnError(RuntimeError):
@@ -69,16 +74,20 @@ def lib():
         L.sattn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
         L.sattn_fwd_host.restype = i
         L.sattn_fwd_host.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+        L.sattn_kernel_launches.restype = ctypes.c_ulonglong
+        L.sattn_kernel_launches.argtypes = [i]
+        L.sattn_debug_set_wait_limit.restype = i
+        L.sattn_debug_set_wait_limit.argtypes = [ctypes.c_longlong, i]
         _lib = L
     return _lib
 
 
-def mode_code(mode, dtype):
+def mode_code(mode, dtype, q_per_token=False):
     if mode not in MODES:
         raise ValueError(f"mode must be one of {list(MODES)}")
     if dtype not in (torch.bfloat16, torch.float16):
         raise TypeError("q, k, v must be bfloat16 or float16")
-    return MODES[mode] | (FP16_IO if dtype == torch.float16 else 0)
+    return MODES[mode] | (FP16_IO if dtype == torch.float16 else 0) | (Q_PER_TOKEN if q_per_token else 0)
 
 
 def _check(status, what):
@@ -104,21 +113,22 @@ def _check_qkv(q, k, v):
     return tuple(q.shape)
 
 
-def workspace_bytes(B, H, N, d, mode="i8f8", dtype=torch.bfloat16):
-    return int(lib().sattn_workspace_bytes(B, H, N, d, mode_code(mode, dtype)))
+def workspace_bytes(B, H, N, d, mode="i8f8", dtype=torch.bfloat16, q_per_token=False):
+    return int(lib().sattn_workspace_bytes(B, H, N, d, mode_code(mode, dtype, q_per_token)))
 
 
-def workspace_layout(B, H, N, d, mode="i8f8", dtype=torch.bfloat16):
+def workspace_layout(B, H, N, d, mode="i8f8", dtype=torch.bfloat16, q_per_token=False):
     out = WsLayout()
-    _check(lib().sattn_workspace_layout(B, H, N, d, mode_code(mode, dtype), ctypes.byref(out)),
+    _check(lib().sattn_workspace_layout(B, H, N, d, mode_code(mode, dtype, q_per_token), ctypes.byref(out)),
            "sattn_workspace_layout")
     return {n: getattr(out, n) for n, _ in WsLayout._fields_}
 
 
-def quantize(q, k, v, mode="i8f8", workspace=None, stream=None):
-    """Quantise q, k, v into a uint8 workspace tensor (allocated when not given)."""
+def quantize(q, k, v, mode="i8f8", workspace=None, stream=None, q_per_token=False):
+    """Quantise q, k, v into a uint8 workspace tensor (allocated when not given).
+    ``q_per_token``: one INT8 scale per query token (I8QK_F8PV only)."""
     B, H, N, d = _check_qkv(q, k, v)
-    m = mode_code(mode, q.dtype)
+    m = mode_code(mode, q.dtype, q_per_token)
     nbytes = int(lib().sattn_workspace_bytes(B, H, N, d, m))
     if nbytes == 0:
         raise SattnError(2, "sattn_workspace_bytes")
@@ -131,31 +141,31 @@ def quantize(q, k, v, mode="i8f8", workspace=None, stream=None):
 
 
 def fwd_quantized(workspace, shape, causal=False, sm_scale=None, mode="i8f8", dtype=torch.bfloat16,
-                  out=None, stream=None):
+                  out=None, stream=None, q_per_token=False):
     """Attention over a workspace filled by ``quantize``; returns out [B, H, N, d]."""
     B, H, N, d = shape
     if out is None:
         out = torch.empty((B, H, N, d), dtype=dtype, device=workspace.device)
     _check(lib().sattn_fwd_quantized(workspace.data_ptr(), workspace.numel(), out.data_ptr(),
                                      B, H, N, d, int(bool(causal)), float(sm_scale or 0.0),
-                                     mode_code(mode, dtype), _stream(stream)),
+                                     mode_code(mode, dtype, q_per_token), _stream(stream)),
            "sattn_fwd_quantized")
     return out
 
 
-def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None):
+def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None, q_per_token=False):
     """O = softmax(Q K^T * sm_scale) V with quantised operands (library-owned workspace)."""
     B, H, N, d = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
     _check(lib().sattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
-                           int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype),
+                           int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype, q_per_token),
                            _stream(stream)),
            "sattn_fwd")
     return out
 
 
-def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None):
+def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None, q_per_token=False):
     """``fwd`` on host (CPU) tensors: copies in, computes and copies out chunk by
     chunk, overlapping the transfers with the compute.  Pinned tensors
     (``tensor.pin_memory()``) let the copies run asynchronously.  The call is
@@ -174,7 +184,7 @@ def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream
     elif out.is_cuda or not out.is_contiguous() or out.shape != q.shape or out.dtype != q.dtype:
         raise ValueError("out must be a contiguous host tensor like q")
     _check(lib().sattn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
-                                int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype),
+                                int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype, q_per_token),
                                 _stream(stream)),
            "sattn_fwd_host")
     return out
@@ -183,3 +193,8 @@ def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream
 def device_error(clear=False):
     """Device-side error word (0 = no bounded wait ran out); synchronises the device."""
     return int(lib().sattn_device_error(int(bool(clear))))
+
+
+def kernel_launches(reset=False):
+    """CUDA kernels the library has launched since load or the last reset."""
+    return int(lib().sattn_kernel_launches(int(bool(reset))))

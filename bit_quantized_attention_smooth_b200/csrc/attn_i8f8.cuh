@@ -5,20 +5,29 @@
 // P V.  Per query tile of 128 rows and key tile j of 128 keys:
 //   S_int  = q8 . k8^T                         tcgen05.mma kind::i8 -> int32 TMEM
 //   S2     = S_int * s_q * s_k[j] * sm_scale * log2(e)
-//   m      = running row max of S2 (online softmax)
+//   m      = reference max of the row (lazy: see below)
 //   P~     = 2^(S2 - m);  l = alpha l + rowsum(P~)   FP32, one row per thread
-//   p8     = E4M3(448 P~)                      -> shared memory
+//   p8     = E4M3(c_P P~),  c_P = 448 * 2^-tau   -> shared memory
 //   O_in  (+)= p8 . v8                         tcgen05.mma kind::f8f6f4 -> fp32 TMEM
+// Lazy reference max: m moves to a tile's row max only when that max exceeds
+// m by more than tau = kLazyTau, so P~ <= 2^tau and c_P maps 2^tau onto 448.
+// Each tile is processed in ONE speculative pass over S with the current m,
+// which also tracks the row's largest exponent argument; only when some row
+// of the warp went more than tau above its m (rare after the first tile) does
+// the warp take the tile's row max from that argument and redo its P rows.
+// The first tile is a pass against m = 0 (only its maximum is used) and a redo.
 // Two-level accumulation: the tensor cores accumulate O_in over a group of
 // kFlushEvery key tiles; at the start of every group the softmax threads add
 // O_in into the outer FP32 accumulator O_out (registers) and the next P V
-// overwrites O_in.  When a row's running max grows, O_out is rescaled by
+// overwrites O_in.  When a row's reference max moves, O_out is rescaled by
 // alpha = 2^(m_old - m_new) through a per-row factor (O_out = beta * o_out,
 // beta *= alpha), and inside a group that row's O_in in TMEM is multiplied by
 // alpha (per warp, only when some lane of the warp needs it).  Both happen
 // after P of the tile has been written, when the previous P V has long
 // completed.  Finally
-//   O = (O_out + O_in) * s_v[c] / (448 l).
+//   O = (O_out + O_in) * s_v[c] / (c_P l).
+// Q scales: one per 128-token tile, or one per token (the row's thread holds
+// its own scale, so the finer granularity costs nothing here).
 //
 // CTA = two 128-row query tiles (A, B) of one (b, h) sharing every K/V tile;
 // 12 warps in 3 warpgroups:
@@ -30,15 +39,16 @@
 //              the softmax warpgroups through setmaxnreg)
 // Two softmax warps per SM sub-partition hide each other's latency.  TMEM
 // columns: S_A [0,128), S_B [128,256), O_in_A [256,256+D), O_in_B
-// [256+D, 256+2D).  Each softmax warp reads its S twice (row max, then P),
-// 64 columns at a time (two 32-column loads behind one wait), so that the 128
-// outer-accumulator registers and the 64 score registers fit in the softmax
-// warps' 232.
+// [256+D, 256+2D).  Each softmax warp reads its S once per tile (twice at
+// the first tile and when it redoes one), 64 columns at a time (two 32-column loads behind one
+// wait), so that the 128 outer-accumulator registers and the 64 score
+// registers fit in the softmax warps' 232.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "../../include/sattn.h"
 #include "ptx.cuh"
 
 namespace sattn {
@@ -54,14 +64,20 @@ constexpr int kControlRegs = 40;        // per thread, warpgroup 2 (TMA, MMA, 2 
 // fit in what the block was launched with (threads x launch registers).
 constexpr int kRegsNeeded = 256 * kSoftmaxRegs + 128 * kControlRegs;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
+// Lazy reference max threshold (log2 units) and the static FP8 scale of P it
+// implies: c_P = 448 * 2^-tau, log2(c_P) = log2(448) - tau.
+constexpr float kLazyTau = SATTN_I8F8_LAZY_TAU;
+constexpr float kLog2_CP = kLog2_448 - kLazyTau;
 
 struct AttnArgs {
-  const float *sq;   // [BH, nblk]
+  const float *sq;   // [BH, sq_stride]: per 128-token tile (nblk) or per token (N)
   const float *sk;   // [BH, nblk]
   const float *sv;   // [BH, D]
   void *out;         // [BH, N, D] bf16 / fp16
   int N;
   int nblk;          // ceil(N / 128)
+  int sq_stride;     // nblk, or N when q_per_token
+  int q_per_token;   // 1: one Q scale per token
   float sm_log2;     // sm_scale * log2(e)
 };
 
@@ -100,13 +116,6 @@ __device__ __forceinline__ uint32_t pack2_out<__half>(float a, float b) {
 // Sentinel for a masked score; |q8 . k8| <= 127 * 127 * 128 < 2^22, so no
 // real INT8 score takes this value.
 constexpr uint32_t kMaskedScore = 0x80000000u;
-// int32 -> float without a conversion instruction: for |s| < 2^22 the float
-// with bits (s + 0x4B400000) equals 12582912 + s exactly.  The exponent
-// argument 2^(s c - m') is then one FMA: (12582912 + s) c - (12582912 c + m').
-// Rounding the constant costs at most c/2 in the exponent, i.e. half of one
-// integer score step, far below the INT8 quantisation error of the scores.
-constexpr int kMagicI = 0x4B400000;
-constexpr float kMagicF = 12582912.0f;
 
 __device__ __forceinline__ void mask_chunk(uint32_t (&s)[32], int kv0, int N, bool causal, int row_g) {
 #pragma unroll
@@ -129,30 +138,37 @@ __device__ __forceinline__ int tree_max32(const uint32_t (&s)[32]) {
   return m[0];
 }
 
-// 32 scores -> 32 E4M3 codes of 448 P~ (two 16-byte chunks of the row's
+// 32 scores -> 32 E4M3 codes of c_P P~ (two 16-byte chunks of the row's
 // 128-byte line in the 128-byte-swizzled K-major layout the MMA reads:
 // 16-byte chunk c of row r lives at chunk c ^ (r mod 8)); accumulates the
-// unquantised 448 P~ into sum2 (two partial sums).
-// b = 12582912 c + (m - log2 448).
-template <bool MASKED>
+// unquantised c_P P~ into sum2 (two partial sums) and, with TRACK, the
+// largest exponent argument x = S2 - m + log2 c_P into xmax2.
+// x = float(s) c - b with b = m - log2 c_P: the int32 -> float conversion is
+// exact (|s| < 2^22) and x is one FMA, so it is within half an ulp; E4M3
+// codes of P then agree with an exact computation except at rounding ties.
+template <bool MASKED, bool TRACK>
 __device__ __forceinline__ void p_chunk(const uint32_t (&s)[32], float c, float b, uint8_t *prow, int c16, int r,
-                                        float2 &sum2) {
+                                        float2 &sum2, float2 &xmax2) {
   const float2 c2 = make_float2(c, c);
   const float2 nb2 = make_float2(-b, -b);
   uint32_t w[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    float2 x01 = ffma2(make_float2(__int_as_float(static_cast<int>(s[4 * q]) + kMagicI),
-                                   __int_as_float(static_cast<int>(s[4 * q + 1]) + kMagicI)),
+    float2 x01 = ffma2(make_float2(static_cast<float>(static_cast<int>(s[4 * q])),
+                                   static_cast<float>(static_cast<int>(s[4 * q + 1]))),
                        c2, nb2);
-    float2 x23 = ffma2(make_float2(__int_as_float(static_cast<int>(s[4 * q + 2]) + kMagicI),
-                                   __int_as_float(static_cast<int>(s[4 * q + 3]) + kMagicI)),
+    float2 x23 = ffma2(make_float2(static_cast<float>(static_cast<int>(s[4 * q + 2])),
+                                   static_cast<float>(static_cast<int>(s[4 * q + 3]))),
                        c2, nb2);
     if (MASKED) {
       if (s[4 * q] == kMaskedScore) x01.x = -INFINITY;
       if (s[4 * q + 1] == kMaskedScore) x01.y = -INFINITY;
       if (s[4 * q + 2] == kMaskedScore) x23.x = -INFINITY;
       if (s[4 * q + 3] == kMaskedScore) x23.y = -INFINITY;
+    }
+    if (TRACK) {
+      xmax2.x = fmax3(xmax2.x, x01.x, x01.y);
+      xmax2.y = fmax3(xmax2.y, x23.x, x23.y);
     }
     const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
     const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
@@ -161,6 +177,32 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&s)[32], float c, float 
   }
   *reinterpret_cast<uint4 *>(prow + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   *reinterpret_cast<uint4 *>(prow + (((c16 + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// One pass over an S tile: P~ codes of the row into its P line in shared
+// memory; returns the row's sum of c_P P~ and (into xmax2) its largest
+// exponent argument x = S2 - m + log2 c_P.
+__device__ __forceinline__ float p_pass(uint32_t s_tmem, float c, float b, uint8_t *prow, int r, bool masked, int kv0,
+                                        int N, bool causal, int row_g, float2 &xmax2) {
+  float2 tsum2 = make_float2(0.f, 0.f);
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t s0[32], s1[32];
+    tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
+    tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
+    tmem_ld_wait(s0);
+    tmem_ld_wait(s1);
+    if (masked) {
+      mask_chunk(s0, kv0 + hh * 64, N, causal, row_g);
+      mask_chunk(s1, kv0 + hh * 64 + 32, N, causal, row_g);
+      p_chunk<true, true>(s0, c, b, prow, hh * 4, r, tsum2, xmax2);
+      p_chunk<true, true>(s1, c, b, prow, hh * 4 + 2, r, tsum2, xmax2);
+    } else {
+      p_chunk<false, true>(s0, c, b, prow, hh * 4, r, tsum2, xmax2);
+      p_chunk<false, true>(s1, c, b, prow, hh * 4 + 2, r, tsum2, xmax2);
+    }
+  }
+  return tsum2.x + tsum2.y;
 }
 
 template <int D, bool CAUSAL, typename OutT>
@@ -245,6 +287,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       int last_j = -1;
+      const int withheld = g_withhold_k_tile;            // -1 except under the failure-path test hook
       const int nq = nkv_of[1] > 0 ? 2 : 1;             // tile B may lie past the last token
       mbar_arrive_expect_tx(q_full, nq * L::kQBytes);
       for (int x = 0; x < nq; ++x)
@@ -253,10 +296,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int s = j % kKVStages;
         const uint32_t ph = (j / kKVStages) & 1;
         if (!mbar_wait(&k_empty[s], ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&k_full[s], L::kKBytes);
-        tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
+        if (j != withheld) {
+          mbar_arrive_expect_tx(&k_full[s], L::kKBytes);
+          tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
+        }
         if (!mbar_wait(&v_empty[s], ph ^ 1, abort_flag)) {
-          drain_wait(&k_full[s], ph);   // K_j is in flight without its V_j
+          if (j != withheld) drain_wait(&k_full[s], ph);   // K_j is in flight without its V_j
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kVBytes);
@@ -268,7 +313,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         drain_wait(q_full, 0);
         for (int j = max(0, last_j - kKVStages + 1); j <= last_j; ++j) {
           const uint32_t ph = (j / kKVStages) & 1;
-          drain_wait(&k_full[j % kKVStages], ph);
+          if (j != withheld) drain_wait(&k_full[j % kKVStages], ph);
           drain_wait(&v_full[j % kKVStages], ph);
         }
       }
@@ -346,15 +391,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t s_tmem = tmem + lane_base + x * kTile;
     const uint32_t o_tmem = tmem + lane_base + kOin0 + x * D;
     const int row_g = qt * kTile + r;
-    const float cq = nkv > 0 ? args.sq[static_cast<size_t>(bh) * args.nblk + qt] * args.sm_log2 : 0.f;
+    const int sq_idx = args.q_per_token ? min(row_g, N - 1) : qt;
+    const float cq = nkv > 0 ? args.sq[static_cast<size_t>(bh) * args.sq_stride + sq_idx] * args.sm_log2 : 0.f;
     const float *sk = args.sk + static_cast<size_t>(bh) * args.nblk;
     uint8_t *p_base = smem + L::kP + (x * 2) * L::kPBytes + r * 128;
 
     float o_out[D];
 #pragma unroll
     for (int i = 0; i < D; ++i) o_out[i] = 0.f;
-    float m_ref = -INFINITY;
-    float l448 = 0.f;          // sum of 448 * P~ (the static FP8 scale folded in)
+    float m_ref = -INFINITY;   // reference max of the row (lazy)
+    float lsum = 0.f;          // sum of c_P * P~ (the static FP8 scale folded in)
     float beta = 1.f;          // the outer accumulator is beta * o_out (rescaled lazily)
     bool ok = true;
 
@@ -362,61 +408,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!mbar_wait(&s_full[x], j & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const bool masked = ((j == nkv_all - 1) && (N & (kTile - 1))) || (CAUSAL && j == qt);
-
-      // pass 1: row max of the integer scores (a rolled loop over two 64-column
-      // halves, each read with two loads behind one wait, keeps the loop body
-      // small enough for the instruction cache)
-      int smax = INT_MIN;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        // two 32-column loads behind one wait: one TMEM round trip per 64 columns
-        uint32_t s0[32], s1[32];
-        tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
-        tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
-        tmem_ld_wait(s0);
-        tmem_ld_wait(s1);
-        if (masked) {
-          mask_chunk(s0, j * kTile + hh * 64, N, CAUSAL, row_g);
-          mask_chunk(s1, j * kTile + hh * 64 + 32, N, CAUSAL, row_g);
-        }
-        smax = max(smax, max(tree_max32(s0), tree_max32(s1)));
-      }
+      const int kv0 = j * kTile;
       const float c = cq * sk[j];
-      const float m_new = fmaxf(m_ref, static_cast<float>(smax) * c);
-      const float alpha = ex2_approx(m_ref - m_new);    // 0 at the first tile (m_ref = -inf)
-      const float bconst = fmaf(kMagicF, c, m_new - kLog2_448);
 
-      // pass 2: P~ -> E4M3 into P buffer (j & 1), once P V of tile j-2 has read it
+      // P~ -> E4M3 into P buffer (j & 1), once P V of tile j-2 has read it
       const int pb = x * 2 + (j & 1);
       if (!mbar_wait(&pv_done[pb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       uint8_t *prow = p_base + (j & 1) * L::kPBytes;
-      float2 tsum2 = make_float2(0.f, 0.f);
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t s0[32], s1[32];
-        tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
-        tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
-        tmem_ld_wait(s0);
-        tmem_ld_wait(s1);
-        if (masked) {
-          mask_chunk(s0, j * kTile + hh * 64, N, CAUSAL, row_g);
-          mask_chunk(s1, j * kTile + hh * 64 + 32, N, CAUSAL, row_g);
-          p_chunk<true>(s0, c, bconst, prow, hh * 4, r, tsum2);
-          p_chunk<true>(s1, c, bconst, prow, hh * 4 + 2, r, tsum2);
-        } else {
-          p_chunk<false>(s0, c, bconst, prow, hh * 4, r, tsum2);
-          p_chunk<false>(s1, c, bconst, prow, hh * 4 + 2, r, tsum2);
-        }
+      // speculative pass with the current reference max (0 at the first tile,
+      // which only serves to find the tile's row max)
+      const float m_try = j > 0 ? m_ref : 0.f;
+      float2 xm2 = make_float2(-INFINITY, -INFINITY);
+      float tsum = p_pass(s_tmem, c, m_try - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
+      // x = S2 - m + log2 c_P;  the row max moves when S2max - m > tau  <=>  xmax > log2 448
+      const float xmax = fmaxf(xm2.x, xm2.y);
+      const bool up = j == 0 || xmax > kLog2_448;
+      const bool moved = __any_sync(0xffffffffu, up);   // warp-uniform
+      float m_new = m_ref, alpha = 1.f;
+      if (moved) {
+        if (up) m_new = fmaxf(m_ref, xmax + (m_try - kLog2_CP));   // the tile's row max
+        alpha = j > 0 ? ex2_approx(m_ref - m_new) : 0.f;
+        tsum = p_pass(s_tmem, c, m_new - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
       }
-      const float tsum = tsum2.x + tsum2.y;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[x]);
-      l448 = fmaf(alpha, l448, tsum);
+      lsum = fmaf(alpha, lsum, tsum);
 
-      // two-level accumulation: flush O_in at a group start, or rescale on a max increase
+      // two-level accumulation: flush O_in at a group start, or rescale when the reference max moved
       const bool boundary = j > 0 && (j % kFlushEvery) == 0;
-      const bool grow = __any_sync(0xffffffffu, j > 0 && m_new > m_ref);
+      const bool grow = j > 0 && moved;
       if (boundary || grow) {
         const int t = j - 1;
         if (!mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -476,7 +497,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int t = nkv - 1;
       if (mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) {
         tc_fence_after();
-        const float inv_l = 1.f / l448;
+        const float inv_l = 1.f / lsum;
         const float *sv = args.sv + static_cast<size_t>(bh) * D;
         OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D;
 #pragma unroll

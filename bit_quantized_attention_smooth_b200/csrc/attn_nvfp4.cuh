@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       int last_j = -1;
+      const int withheld = g_withhold_k_tile;            // -1 except under the failure-path test hook
       const size_t sf_qk_tile = static_cast<size_t>(L::kSfQK);
       mbar_arrive_expect_tx(q_full, L::kQBytes + L::kSfQK);
       tma_load_3d(smem + L::kQ, &tm_q, q_full, 0, qt * kTile, bh);
@@ -223,12 +224,14 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         const int s = j % kKVStages;
         const uint32_t ph = (j / kKVStages) & 1;
         if (!mbar_wait(&k_empty[s], ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&k_full[s], L::kKBytes + L::kSfQK);
-        tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
-        bulk_load(smem + L::kSfK + s * L::kSfQK, args.sfk + (static_cast<size_t>(bh) * nkv_all + j) * sf_qk_tile,
-                  L::kSfQK, &k_full[s]);
+        if (j != withheld) {
+          mbar_arrive_expect_tx(&k_full[s], L::kKBytes + L::kSfQK);
+          tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
+          bulk_load(smem + L::kSfK + s * L::kSfQK, args.sfk + (static_cast<size_t>(bh) * nkv_all + j) * sf_qk_tile,
+                    L::kSfQK, &k_full[s]);
+        }
         if (!mbar_wait(&v_empty[s], ph ^ 1, abort_flag)) {
-          drain_wait(&k_full[s], ph);
+          if (j != withheld) drain_wait(&k_full[s], ph);
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kVBytes + L::kSfV);
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         drain_wait(q_full, 0);
         for (int j = max(0, last_j - kKVStages + 1); j <= last_j; ++j) {
           const uint32_t ph = (j / kKVStages) & 1;
-          drain_wait(&k_full[j % kKVStages], ph);
+          if (j != withheld) drain_wait(&k_full[j % kKVStages], ph);
           drain_wait(&v_full[j % kKVStages], ph);
         }
       }

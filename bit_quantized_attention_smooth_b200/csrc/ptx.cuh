@@ -19,6 +19,14 @@ constexpr unsigned kErrWaitTimeout = 1u;
 constexpr long long kWaitLimitCycles = 4000000000ll;
 constexpr uint32_t kWaitCheckEvery = 256;
 
+// Runtime bound of the role waits (mbar_wait); drain waits keep the constant
+// kWaitLimitCycles so that copies and MMAs already in flight always complete.
+// Lowered only by the failure-path test hook (sattn_debug_set_wait_limit).
+__device__ long long g_wait_limit = kWaitLimitCycles;
+// Failure-path test hook: when >= 0, the TMA producers never load this key
+// tile (its barrier then never completes and the waits for it run out).
+__device__ int g_withhold_k_tile = -1;
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -50,7 +58,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits until the phase with parity `parity` of `bar` has completed.  Gives up
-// after kWaitLimitCycles or when `abort_flag` (CTA shared) becomes non-zero;
+// after g_wait_limit cycles or when `abort_flag` (CTA shared) becomes non-zero;
 // on time-out it records kErrWaitTimeout in g_error_word and raises the abort
 // flag so that every role of the CTA leaves its loop.  Returns false when it
 // gave up.
@@ -61,7 +69,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((i % kWaitCheckEvery) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > g_wait_limit) {
         atomicOr(&g_error_word, kErrWaitTimeout);
         *abort_flag = 1;
         return false;
@@ -308,6 +316,15 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "=l"(d)
       : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
   return *reinterpret_cast<float2 *>(&d);
+}
+
+// Maximum that propagates NaN (fmaxf drops it): the quantisers' scales use it so
+// that a NaN input turns the scale it feeds, and the outputs that use that
+// scale, into NaN.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
 // Maximum of three floats in one instruction.

@@ -5,15 +5,25 @@
 // outlier smoothing; the SageAttention tag page (reportify.cn), SageAttention3
 // summary, bullet [17], quantises Q/K per block.  Readings used here:
 //   mu[c]   = (float)( sum_n K[n,c] (exact float64 sum) / N )      per (b,h)
-//   s_q, s_k = max|x| / 127 per 128-token block (1 for an all-zero block)
+//   s_q, s_k = max|x| / 127 per 128-token block (1 for an all-zero block);
+//             optionally s_q per token (max over the token's channels)
 //   q8      = RNE(x / s) clamped to [-127, 127], division in IEEE float32
 //   s_v[c]  = max_n |V[n,c]| / 448 per channel (1 for an all-zero channel)
 //   v8      = E4M3_RNE_satfinite(V / s_v), written transposed [d, Nv]
 //
+// NaN inputs: every maximum above propagates NaN (fmax_nan), so a NaN makes
+// the scale it feeds NaN: a Q block's (or token's) rows, a K channel's mean
+// (and with it every K scale of the head), a V channel's scale.
+//
 // HBM-bound.  Pass 1 (kv_stats) reads K and V once and reduces per-channel
-// sums (float64 atomics: exact for bf16/fp16 inputs, so order-independent)
-// and per-channel |V| maxima.  Pass 2 reads Q, K, V once more and writes the
-// codes; every load is a coalesced 16-byte vector.
+// sums in float64 atomics and per-channel |V| maxima.  Each bf16/fp16 value is
+// exact in float64, and so is every partial sum while the sum's magnitude
+// stays below 2^53 times the smallest quantum among the summands (true for
+// the workloads here: values above 2^-30 in magnitude, sums below 2^21), so
+// the mean does not depend on the order of the atomics; a head holding values
+// as small as fp16/bf16 subnormals next to sums near 2^30 can differ in the
+// mean's last bit between runs.  Pass 2 reads Q, K, V once more and writes
+// the codes; every load is a coalesced 16-byte vector.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -90,7 +100,7 @@ __global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__rest
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       acc[i] += static_cast<double>(kf[i]);
-      vm[i] = fmaxf(vm[i], fabsf(vf[i]));
+      vm[i] = fmax_nan(vm[i], fabsf(vf[i]));
     }
   }
 #pragma unroll
@@ -105,7 +115,7 @@ __global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__rest
     float m = 0.f;
     for (int r = 0; r < RPI; ++r) {
       s += s_sum[r][c];
-      m = fmaxf(m, s_max[r][c]);
+      m = fmax_nan(m, s_max[r][c]);
     }
     atomicAdd(ksum + static_cast<size_t>(bh) * D + c, s);
     atomicMax(vmax + static_cast<size_t>(bh) * D + c, __float_as_uint(m));  // m >= 0: bit order = value order
@@ -115,13 +125,13 @@ __global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__rest
 template <int NT>
 __device__ __forceinline__ float block_max(float v, float *s_red) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  for (int o = 16; o > 0; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(0xffffffffu, v, o));
   const int warp = threadIdx.x >> 5;
   if ((threadIdx.x & 31) == 0) s_red[warp] = v;
   __syncthreads();
   float m = s_red[0];
 #pragma unroll
-  for (int w = 1; w < NT / 32; ++w) m = fmaxf(m, s_red[w]);
+  for (int w = 1; w < NT / 32; ++w) m = fmax_nan(m, s_red[w]);
   return m;
 }
 
@@ -172,14 +182,14 @@ __global__ void __launch_bounds__(kBlockQuantThreads, 2) quant_qk_kernel(const T
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         val[it][i] = valid ? __fsub_rn(val[it][i], mu[i]) : 0.f;
-        amax = fmaxf(amax, fabsf(val[it][i]));
+        amax = fmax_nan(amax, fabsf(val[it][i]));
       }
     }
   } else {
 #pragma unroll
     for (int it = 0; it < ITERS; ++it)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(val[it][i]));
+      for (int i = 0; i < 8; ++i) amax = fmax_nan(amax, fabsf(val[it][i]));
   }
   amax = block_max<kBlockQuantThreads>(amax, s_red);
   const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
@@ -189,6 +199,59 @@ __global__ void __launch_bounds__(kBlockQuantThreads, 2) quant_qk_kernel(const T
   for (int it = 0; it < ITERS; ++it) {
     const int n = blk * kBlockTokens + it * RPI + r0;
     if (n < N) {
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int qi = __float2int_rn(__fdiv_rn(val[it][i], s));
+        qi = max(-127, min(127, qi));
+        w[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
+      }
+      *reinterpret_cast<uint2 *>(out + head + static_cast<size_t>(n) * D + cg * 8) = make_uint2(w[0], w[1]);
+    }
+  }
+}
+
+// Pass 2a, per-token variant: INT8 of Q with one scale per token ("thread-level"
+// granularity: the attention kernel gives each query row its own thread), s =
+// max|x[n, :]| / 127.  grid (ceil(N / kTokRows), B*H), block kQuantThreads;
+// D/8 consecutive lanes share a token (8 channels each) and every thread takes
+// kTokIters tokens, loaded before any is reduced.
+constexpr int kTokIters = 4;
+template <int D>
+__host__ __device__ constexpr int tok_rows_per_cta() { return kQuantThreads / (D / 8) * kTokIters; }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kQuantThreads) quant_q_token_kernel(const T *__restrict__ x, int8_t *__restrict__ out,
+                                                                      float *__restrict__ scale, int N) {
+  constexpr int LPR = D / 8;                  // lanes per token (16 or 8); divides 32
+  constexpr int RPI = kQuantThreads / LPR;    // tokens per iteration of the CTA
+  const int bh = blockIdx.y;
+  const int cg = threadIdx.x % LPR;
+  const size_t head = static_cast<size_t>(bh) * N * D;
+  const int n0 = blockIdx.x * tok_rows_per_cta<D>() + threadIdx.x / LPR;
+  float val[kTokIters][8];
+#pragma unroll
+  for (int it = 0; it < kTokIters; ++it) {
+    const int n = n0 + it * RPI;
+    if (n < N) {
+      load8<T>(x + head + static_cast<size_t>(n) * D + cg * 8, val[it]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) val[it][i] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int it = 0; it < kTokIters; ++it) {
+    const int n = n0 + it * RPI;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmax_nan(amax, fabsf(val[it][i]));
+    // every lane of the warp takes part (tokens past N hold zeros)
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+    if (n < N) {
+      if (cg == 0) scale[static_cast<size_t>(bh) * N + n] = s;
       uint32_t w[2] = {0u, 0u};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {

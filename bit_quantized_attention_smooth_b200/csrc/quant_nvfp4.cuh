@@ -55,7 +55,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t nvfp4_block(const float (&x)[16], uint32_t (&w)[2]) {
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  for (int i = 0; i < 16; ++i) amax = fmax_nan(amax, fabsf(x[i]));
   const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
   const float sc = e4m3_to_float(sc_code);
   w[0] = w[1] = 0u;

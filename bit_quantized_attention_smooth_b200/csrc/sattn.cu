@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <algorithm>
 #include <cmath>
@@ -24,14 +25,24 @@ constexpr int kMaxDevices = 64;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Kernels this library has launched since load (or the last reset).
+std::atomic<unsigned long long> g_launches{0};
+
+constexpr int kFlagBits = SATTN_FP16_IO | SATTN_Q_PER_TOKEN;
+
+int base_mode(int mode) { return mode & ~kFlagBits; }
+
 bool valid_mode(int mode) {
-  const int base = mode & ~SATTN_FP16_IO;
-  return (mode & ~(SATTN_FP16_IO | 0xFF)) == 0 && (base == SATTN_I8QK_F8PV || base == SATTN_NVFP4);
+  const int base = base_mode(mode);
+  return (mode & ~(kFlagBits | 0xFF)) == 0 && (base == SATTN_I8QK_F8PV || base == SATTN_NVFP4);
 }
+
+bool q_per_token(int mode) { return (mode & SATTN_Q_PER_TOKEN) != 0; }
 
 int check_shape(int B, int H, int N, int d, int mode) {
   if (B < 1 || H < 1 || N < 1) return SATTN_ERR_INVALID_ARG;
   if (!valid_mode(mode)) return SATTN_ERR_INVALID_ARG;
+  if (q_per_token(mode) && base_mode(mode) != SATTN_I8QK_F8PV) return SATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return SATTN_ERR_UNSUPPORTED;
   const long long total = static_cast<long long>(B) * H * N * d;
   if (total >= (1LL << 31) || static_cast<long long>(B) * H >= 65536) return SATTN_ERR_UNSUPPORTED;
@@ -40,7 +51,7 @@ int check_shape(int B, int H, int N, int d, int mode) {
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool is_nvfp4(int mode) { return (mode & ~SATTN_FP16_IO) == SATTN_NVFP4; }
+bool is_nvfp4(int mode) { return base_mode(mode) == SATTN_NVFP4; }
 
 // NVFP4 workspace: q8/k8/vt8 hold the packed E2M1 codes of Q, K - mean and
 // V^T (N rounded up to 32 tokens), sq/sk/sv the E4M3 scale blocks of Q, K, V.
@@ -64,7 +75,9 @@ sattn_ws_layout_t make_layout_nvfp4(int B, int H, int N, int d) {
   return L;
 }
 
-sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d) {
+// I8F8 workspace; with per-token Q scales, sq holds N floats per head instead
+// of one per 128-token block.
+sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d, bool per_token) {
   sattn_ws_layout_t L;
   std::memset(&L, 0xFF, sizeof(L));
   const size_t BH = static_cast<size_t>(B) * H;
@@ -74,7 +87,7 @@ sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d) {
   L.q8 = off;   off = align_up(off + BH * N * d, kSectionAlign);
   L.k8 = off;   off = align_up(off + BH * N * d, kSectionAlign);
   L.vt8 = off;  off = align_up(off + BH * d * L.nv, kSectionAlign);
-  L.sq = off;   off = align_up(off + BH * L.nblk * sizeof(float), kSectionAlign);
+  L.sq = off;   off = align_up(off + BH * (per_token ? N : L.nblk) * sizeof(float), kSectionAlign);
   L.sk = off;   off = align_up(off + BH * L.nblk * sizeof(float), kSectionAlign);
   L.sv = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
@@ -85,7 +98,7 @@ sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d) {
 }
 
 sattn_ws_layout_t make_layout(int B, int H, int N, int d, int mode) {
-  return is_nvfp4(mode) ? make_layout_nvfp4(B, H, N, d) : make_layout_i8f8(B, H, N, d);
+  return is_nvfp4(mode) ? make_layout_nvfp4(B, H, N, d) : make_layout_i8f8(B, H, N, d, q_per_token(mode));
 }
 
 // ---------------------------------------------------------------- tensor maps
@@ -122,7 +135,7 @@ bool make_map_u8(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim
 
 template <typename T, int D>
 int launch_quant_i8f8(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws,
-                      const sattn_ws_layout_t &L, cudaStream_t st) {
+                      const sattn_ws_layout_t &L, bool per_token, cudaStream_t st) {
   double *ksum = reinterpret_cast<double *>(ws + L.ksum);
   unsigned *vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
   if (cudaMemsetAsync(ws + L.ksum, 0, L.total - L.ksum, st) != cudaSuccess) return SATTN_ERR_CUDA;
@@ -130,14 +143,21 @@ int launch_quant_i8f8(const void *q, const void *k, const void *v, int BH, int N
   kv_stats_kernel<T, D><<<dim3((N + tpc - 1) / tpc, BH), kQuantThreads, 0, st>>>(
       static_cast<const T *>(k), static_cast<const T *>(v), ksum, vmax, N, tpc);
   const dim3 grid(L.nblk, BH);
-  quant_qk_kernel<T, D, false><<<grid, kBlockQuantThreads, 0, st>>>(
-      static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq),
-      nullptr, nullptr, N, L.nblk);
+  if (per_token) {
+    const int rows = tok_rows_per_cta<D>();
+    quant_q_token_kernel<T, D><<<dim3((N + rows - 1) / rows, BH), kQuantThreads, 0, st>>>(
+        static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq), N);
+  } else {
+    quant_qk_kernel<T, D, false><<<grid, kBlockQuantThreads, 0, st>>>(
+        static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq),
+        nullptr, nullptr, N, L.nblk);
+  }
   quant_qk_kernel<T, D, true><<<grid, kBlockQuantThreads, 0, st>>>(
       static_cast<const T *>(k), reinterpret_cast<int8_t *>(ws + L.k8), reinterpret_cast<float *>(ws + L.sk), ksum,
       reinterpret_cast<float *>(ws + L.mu), N, L.nblk);
   quant_v_kernel<T, D><<<grid, 4 * D, 0, st>>>(static_cast<const T *>(v), ws + L.vt8,
                                                         reinterpret_cast<float *>(ws + L.sv), vmax, N, L.nv);
+  g_launches += 4;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
@@ -157,6 +177,7 @@ int launch_quant_nvfp4(const void *q, const void *k, const void *v, int BH, int 
   quant_rows_nvfp4_kernel<T, D, true><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(k), ws + L.k8, ws + L.sk,
                                                                       ksum, reinterpret_cast<float *>(ws + L.mu), N);
   quant_v_nvfp4_kernel<T, D><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(v), ws + L.vt8, ws + L.sv, N, L.nv);
+  g_launches += 4;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
@@ -187,12 +208,13 @@ int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, 
   a.nblk = L.nblk;
   a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
   kern<<<dim3(L.nblk, BH), kF4Threads, smem, st>>>(tq, tk, tv, a);
+  g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
 template <int D, bool CAUSAL, typename OutT>
 int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
-                     cudaStream_t st) {
+                     bool per_token, cudaStream_t st) {
   using SL = AttnSmem<D>;
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle swqk = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -219,19 +241,23 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
   a.out = out;
   a.N = N;
   a.nblk = L.nblk;
+  a.sq_stride = per_token ? N : L.nblk;
+  a.q_per_token = per_token ? 1 : 0;
   a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
   kern<<<dim3((L.nblk + kQTiles - 1) / kQTiles, BH), kAttnThreads, smem, st>>>(tq, tk, tv, a);
+  g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
 template <int D, typename OutT>
 int dispatch_attn(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, int causal, float sm,
-                  bool nvfp4, cudaStream_t st) {
-  if (nvfp4)
+                  int mode, cudaStream_t st) {
+  if (is_nvfp4(mode))
     return causal ? launch_attn_nvfp4<D, true, OutT>(ws, L, out, BH, N, sm, st)
                   : launch_attn_nvfp4<D, false, OutT>(ws, L, out, BH, N, sm, st);
-  return causal ? launch_attn_i8f8<D, true, OutT>(ws, L, out, BH, N, sm, st)
-                : launch_attn_i8f8<D, false, OutT>(ws, L, out, BH, N, sm, st);
+  const bool pt = q_per_token(mode);
+  return causal ? launch_attn_i8f8<D, true, OutT>(ws, L, out, BH, N, sm, pt, st)
+                : launch_attn_i8f8<D, false, OutT>(ws, L, out, BH, N, sm, pt, st);
 }
 
 // Library-owned workspace of sattn_fwd, one per device.
@@ -281,11 +307,12 @@ int sattn_quantize(const void *q, const void *k, const void *v, int B, int H, in
     return fp16 ? launch_quant_nvfp4<__half, 64>(q, k, v, BH, N, ws, L, cs)
                 : launch_quant_nvfp4<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, cs);
   }
+  const bool pt = q_per_token(mode);
   if (d == 128)
-    return fp16 ? launch_quant_i8f8<__half, 128>(q, k, v, BH, N, ws, L, cs)
-                : launch_quant_i8f8<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, cs);
-  return fp16 ? launch_quant_i8f8<__half, 64>(q, k, v, BH, N, ws, L, cs)
-              : launch_quant_i8f8<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, cs);
+    return fp16 ? launch_quant_i8f8<__half, 128>(q, k, v, BH, N, ws, L, pt, cs)
+                : launch_quant_i8f8<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, pt, cs);
+  return fp16 ? launch_quant_i8f8<__half, 64>(q, k, v, BH, N, ws, L, pt, cs)
+              : launch_quant_i8f8<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, pt, cs);
 }
 
 int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B, int H, int N, int d, int causal,
@@ -304,12 +331,11 @@ int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int BH = B * H;
   const bool fp16 = (mode & SATTN_FP16_IO) != 0;
-  const bool f4 = is_nvfp4(mode);
   if (d == 128)
-    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, f4, cs)
-                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, f4, cs);
-  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, f4, cs)
-              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, f4, cs);
+    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, mode, cs)
+                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, mode, cs);
+  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, mode, cs)
+              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, mode, cs);
 }
 
 int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
@@ -489,6 +515,19 @@ const char *sattn_status_string(int status) {
     case SATTN_ERR_CUDA: return "SATTN_ERR_CUDA: CUDA runtime error";
     default: return "unknown sattn status";
   }
+}
+
+int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile) {
+  const long long limit = cycles <= 0 ? kWaitLimitCycles : std::max<long long>(cycles, 1000);
+  if (withhold_k_tile < -1) return SATTN_ERR_INVALID_ARG;
+  if (cudaMemcpyToSymbol(g_wait_limit, &limit, sizeof(limit)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_withhold_k_tile, &withhold_k_tile, sizeof(withhold_k_tile)) != cudaSuccess)
+    return SATTN_ERR_CUDA;
+  return SATTN_OK;
+}
+
+unsigned long long sattn_kernel_launches(int reset) {
+  return reset ? g_launches.exchange(0) : g_launches.load();
 }
 
 int sattn_device_error(int clear) {

@@ -14,8 +14,10 @@
  *
  * computed with quantized operands:
  *   SATTN_I8QK_F8PV : K smoothed by its per-channel token mean; Q and K INT8
- *                     with one float32 scale per 128-token block; V FP8 E4M3
- *                     with one scale per channel; P FP8 E4M3 (static scale 448);
+ *                     with one float32 scale per 128-token block (Q: or per
+ *                     token, SATTN_Q_PER_TOKEN); V FP8 E4M3 with one scale per
+ *                     channel; P FP8 E4M3 with the static scale 448 * 2^-tau
+ *                     of a lazy reference max (SATTN_I8F8_LAZY_TAU);
  *                     P.V accumulated in an inner FP32 accumulator that is
  *                     flushed into an outer FP32 accumulator every few key
  *                     blocks (two-level accumulation).
@@ -57,8 +59,20 @@ typedef struct CUstream_st *sattn_stream_t;
 typedef enum {
   SATTN_I8QK_F8PV = 0,
   SATTN_NVFP4 = 1,
-  SATTN_FP16_IO = 0x100 /* flag: q, k, v, out are fp16 instead of bf16 */
+  SATTN_FP16_IO = 0x100,    /* flag: q, k, v, out are fp16 instead of bf16 */
+  SATTN_Q_PER_TOKEN = 0x200 /* flag, I8QK_F8PV only: one INT8 scale per query
+                               token instead of per 128-token block (the
+                               "thread-level quantization" of the QbitAI
+                               reprint, txrjy.com, SageAttention paragraph);
+                               NVFP4 with it is SATTN_ERR_UNSUPPORTED */
 } sattn_mode_t;
+
+/* Lazy reference-max threshold of the I8QK_F8PV softmax (powers of two): a
+ * row's reference max m moves to a key tile's row max only when that max
+ * exceeds m by more than this, so P~ = 2^(S*log2e - m) <= 2^tau and P is
+ * stored as E4M3(448 * 2^-tau * P~).  The pages do not say when the running
+ * max of the streaming softmax moves; 0 would be the exact running max. */
+#define SATTN_I8F8_LAZY_TAU 4.0f
 
 typedef enum {
   SATTN_OK = 0,
@@ -69,37 +83,55 @@ typedef enum {
 } sattn_status_t;
 
 /* Bytes of workspace that sattn_quantize fills for this problem and mode
- * (0 for invalid arguments).  Depends only on (B, H, N, d, mode). */
+ * (0 for invalid arguments).  Depends only on (B, H, N, d, mode).  Bookkeeping
+ * of this library; no passage of the pages defines it. */
 size_t sattn_workspace_bytes(int B, int H, int N, int d, int mode);
 
 /* Quantize q, k, v into `workspace` (device memory of at least
  * sattn_workspace_bytes(...) bytes, 256-byte aligned, owned by the caller).
  * I8QK_F8PV: per-channel K mean (float64 sum of the stored values / N, rounded
- * once to float32), per-block INT8 codes and scales of Q and of K - mean,
- * per-channel FP8 codes and scales of V (V stored transposed, tokens
- * contiguous).  Asynchronous on `stream`.  The workspace stays valid for any
- * number of sattn_fwd_quantized calls with the same (B, H, N, d, mode). */
+ * once to float32: the "outlier smoothing" of the TurboDiffusion explainer,
+ * section 1), INT8 codes and scales of Q (per 128-token block, or per token
+ * with SATTN_Q_PER_TOKEN) and of K - mean per block (tag page, SageAttention3
+ * summary, bullet [17]: per-block INT8), per-channel FP8 codes and scales of V
+ * (explainer, section 1: PV in FP8; V stored transposed, tokens contiguous).
+ * NVFP4: E2M1 codes with one E4M3 scale per 16 values of Q, K - mean (along
+ * channels) and V (along tokens) (tag page, bullet [15]).  A NaN input makes
+ * the scale it feeds NaN.  Asynchronous on `stream`.  The workspace stays
+ * valid for any number of sattn_fwd_quantized calls with the same
+ * (B, H, N, d, mode).  Errors: see the header overview; nothing is written
+ * when an argument is rejected. */
 int sattn_quantize(const void *q, const void *k, const void *v,
                    int B, int H, int N, int d, int mode,
                    void *workspace, size_t ws_bytes, sattn_stream_t stream);
 
 /* Fused attention over a workspace filled by sattn_quantize with the same
- * (B, H, N, d, mode).  Writes out [B, H, N, d].  `out` must not alias the
- * workspace.  Asynchronous on `stream`. */
+ * (B, H, N, d, mode).  Writes out [B, H, N, d].  I8QK_F8PV: S = Q K^T on the
+ * INT8 tensor cores, online softmax in FP32, P in FP8, P V on the FP8 tensor
+ * cores into an inner accumulator flushed into an outer FP32 one every few key
+ * blocks (TurboDiffusion explainer, section 1: INT8 QK, FP8 PV, two-level
+ * accumulation).  NVFP4: block-scaled FP4 tensor cores for both products, P
+ * quantized in two stages (tag page, SageAttention3 summary, bullets
+ * [15][16]).  `out` must not alias the workspace (SATTN_ERR_INVALID_ARG).
+ * Asynchronous on `stream`. */
 int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out,
                         int B, int H, int N, int d, int causal, float sm_scale,
                         int mode, sattn_stream_t stream);
 
 /* sattn_quantize followed by sattn_fwd_quantized, with a workspace that the
- * library owns: one per device, allocated on first use with cudaMallocAsync on
- * `stream` and grown (never shrunk) when a larger problem arrives.  Calls that
- * share a device must be ordered (same stream, or synchronized), because they
- * share this workspace.  `out` must not alias q, k or v. */
+ * library owns: the one-call, drop-in form of the attention (tag page,
+ * SageAttention3 summary, bullet [5]: plug-and-play; explainer, section 1:
+ * usable in place of FlashAttention).  One workspace per device, allocated on
+ * first use with cudaMallocAsync on `stream` and grown (never shrunk) when a
+ * larger problem arrives.  Calls that share a device must be ordered (same
+ * stream, or synchronized), because they share this workspace.  `out` must
+ * not alias q, k or v (SATTN_ERR_INVALID_ARG). */
 int sattn_fwd(const void *q, const void *k, const void *v, void *out,
               int B, int H, int N, int d, int causal, float sm_scale, int mode,
               sattn_stream_t stream);
 
-/* sattn_fwd on HOST buffers: q, k, v and out are host pointers ([B, H, N, d],
+/* sattn_fwd on HOST buffers (a deployment variant; the pages have no
+ * counterpart): q, k, v and out are host pointers ([B, H, N, d],
  * same element type and layout as sattn_fwd); pinned (page-locked) memory lets
  * the copies run asynchronously, pageable memory works but serializes them.
  * The call splits the B*H heads into up to 12 chunks and pipelines them: chunk c
@@ -148,6 +180,24 @@ int sattn_fwd_noalloc(const void *q, const void *k, const void *v, void *out,
 /* Human-readable name of a status code (static string). */
 const char *sattn_status_string(int status);
 
+/* Failure-path test hook; not for production use.  Sets, on the current
+ * device, the bound of the kernels' waits between their roles (cycles <= 0:
+ * the default of about 2-4 s; otherwise at least 1000 cycles) and, when
+ * withhold_k_tile >= 0, makes every attention kernel skip loading that key
+ * tile, so that the waits for it run out: the kernel then sets bit 0 of the
+ * device error word (sattn_device_error), lets the copies and MMAs already in
+ * flight complete, releases its tensor memory and returns with partial
+ * output.  Waits that only drain work in flight keep the default bound.
+ * Call with (0, -1) to restore normal operation.  Synchronous (it writes two
+ * device variables).  Returns SATTN_ERR_INVALID_ARG for withhold_k_tile < -1. */
+int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile);
+
+/* Number of CUDA kernels this library has launched, in this process, since it
+ * was loaded or since the last call with reset != 0 (which returns the count
+ * and sets it to 0).  Counts launches (of every entry point, all devices), not
+ * completions; memset nodes are not counted.  Never touches the GPU. */
+unsigned long long sattn_kernel_launches(int reset);
+
 /* Device-side error word of the current device: 0 when no kernel wait has run
  * out of time since the last clear.  Synchronizes the device.  clear != 0
  * resets the word to 0 after reading. */
@@ -157,7 +207,8 @@ int sattn_device_error(int clear);
  * quantized operands.  Offsets not used by a mode are set to SIZE_MAX.
  *   I8QK_F8PV: q8  int8   [B*H, N, d]        k8 int8 [B*H, N, d]
  *              vt8 e4m3   [B*H, d, Nv]  (Nv = N rounded up to 16)
- *              sq, sk float32 [B*H, ceil(N/128)]   sv, mu float32 [B*H, d]
+ *              sq float32 [B*H, ceil(N/128)], or [B*H, N] with SATTN_Q_PER_TOKEN
+ *              sk float32 [B*H, ceil(N/128)]   sv, mu float32 [B*H, d]
  *              ksum float64 [B*H, d], vmax uint32 [B*H, d] (scratch)
  *   NVFP4 (same fields, other contents):
  *              q8, k8 E2M1 codes, two per byte (low nibble = even channel)
