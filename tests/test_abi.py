@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sattn.h")
 
 OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
-BF16, FP16, NVFP4 = 0, 0x100, 1
+BF16, FP16, NVFP4, QTOK = 0, 0x100, 1, 0x200
 
 
 @pytest.fixture(scope="module")
@@ -97,7 +97,7 @@ def test_invalid_arguments_rejected_before_launch(L):
     g = L.sattn_fwd
     assert g(p, p, p, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
     assert g(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
-    assert g(p, p, p, mis, 1, 2, 256, 128, 0, 0.0, 0x200, None) == INVALID   # unknown flag
+    assert g(p, p, p, mis, 1, 2, 256, 128, 0, 0.0, 0x400, None) == INVALID   # unknown flag
 
 
 def test_fwd_host_rejects_bad_arguments_before_any_cuda_call(L):
@@ -109,7 +109,8 @@ def test_fwd_host_rejects_bad_arguments_before_any_cuda_call(L):
     assert h(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
     assert h(p, p, p, o, 1, 2, 256, 96, 0, 0.0, BF16, None) == UNSUPPORTED
     assert h(p, p, p, o, 1, 2, 0, 64, 0, 0.0, BF16, None) == INVALID
-    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, 0x200, None) == INVALID     # unknown flag
+    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, 0x400, None) == INVALID     # unknown flag
+    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, NVFP4 | QTOK, None) == UNSUPPORTED
 
 
 def test_fwd_host_binding_rejects_device_or_mismatched_tensors():
@@ -120,3 +121,17 @@ def test_fwd_host_binding_rejects_device_or_mismatched_tensors():
         sattn.fwd_host(q, q, q.half())
     with pytest.raises(ValueError):
         sattn.fwd_host(q, q, q, out=torch.zeros(1, 2, 64, 32, dtype=torch.bfloat16))
+
+
+def test_lazy_tau_of_binding_matches_header():
+    m = re.search(r"#define\s+SATTN_I8F8_LAZY_TAU\s+([0-9.]+)f?", open(HEADER).read())
+    assert m and float(m.group(1)) == sattn.I8F8_LAZY_TAU
+
+
+def test_per_token_q_layout(L):
+    blk = sattn.workspace_layout(2, 3, 1000, 128)
+    tok = sattn.workspace_layout(2, 3, 1000, 128, q_per_token=True)
+    assert tok["sk"] - tok["sq"] >= 6 * 1000 * 4 > blk["sk"] - blk["sq"]
+    assert tok["total"] == L.sattn_workspace_bytes(2, 3, 1000, 128, QTOK)
+    assert L.sattn_workspace_bytes(2, 3, 1000, 128, NVFP4 | QTOK) == 0
+    assert L.sattn_workspace_bytes(2, 3, 1000, 128, 0x400) == 0

@@ -2,10 +2,11 @@
 
 Quantiser outputs are compared bit for bit (integer / byte work).  Attention
 outputs are compared element by element with the oracle's emulation of the
-same scheme: max |err| <= 2e-2 and mean |err| <= 2e-3, and with the exact
-float64 attention by cosine similarity (>= 0.999, or no worse than the
-emulation itself by 5e-4 on inputs where the scheme's own accuracy is lower:
-the 0.1 %-outlier workloads).
+same scheme (same lazy reference-max threshold): max |err| <= 2e-2 and
+mean |err| <= 2e-3; and with the exact float64 attention by cosine similarity
+>= 0.999.  On the inputs with 0.1 % x20 Q outliers the scheme itself misses
+0.999 (its emulation does), so the cosine test of those inputs is a strict
+expected failure that records the measured value (see tests/gpu_parity.py).
 """
 
 import numpy as np
@@ -18,10 +19,9 @@ from oracle import attention as A
 from oracle import quant as Qz
 from oracle.formats import e4m3_decode
 import workloads as W
+from tests.gpu_parity import Case, check_cosine_bar, check_parity, miss_params, sample_rows
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS, MEAN_ABS, COS = 2e-2, 2e-3, 0.999
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -86,76 +86,73 @@ def test_quantizer_bit_exact(w):
             assert np.array_equal(e4m3_decode(gv), e4m3_decode(ov))
 
 
-def _check_attention(w, causal, rows=None, heads=None, via_fwd=False):
-    q, k, v = W.make_inputs(w, "cuda")
-    if via_fwd:
-        out = sattn.fwd(q, k, v, causal=causal)
-    else:
-        ws = sattn.quantize(q, k, v)
-        out = sattn.fwd_quantized(ws, q.shape, causal=causal, dtype=q.dtype)
-    torch.cuda.synchronize()
-    if heads is None:
-        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    rows_idx = np.arange(w.N) if rows is None else np.asarray(rows)
-    qf, kf, vf = W.make_heads_f32(w, heads)
-    emu = A.attn_quant_emul_i8f8(qf, kf, vf, causal=causal, rows=rows_idx)
-    exact = A.attn_exact(qf, kf, vf, causal=causal, rows=rows_idx)
-    o = out.float().cpu().numpy()
-    got = np.stack([o[b, h][rows_idx] for (b, h) in heads])
-    err = np.abs(got - emu)
-    cos_gpu, cos_emu = A.cosine(exact, got), A.cosine(exact, emu)
-    print(f"{w.name} causal={causal}: max|err|={err.max():.3e} mean|err|={err.mean():.3e} "
-          f"cos(gpu,exact)={cos_gpu:.6f} cos(emul,exact)={cos_emu:.6f}")
-    assert np.isfinite(got).all()
-    assert err.max() <= MAX_ABS
-    assert err.mean() <= MEAN_ABS
-    assert cos_gpu >= min(COS, cos_emu - 5e-4)
-    return got, emu
-
+OUTLIERS = "0.1 % of Q entries x20: per-{} INT8 Q carries the outliers' scale (emulation cosine {:.5f})"
 
 ATTN_CASES = [
-    (W.SMALL, False),
-    (W.custom(1, 2, 1, 128, seed=11), False),
-    (W.custom(1, 2, 17, 64, "fp16", seed=12), True),
-    (W.custom(1, 3, 127, 128, seed=13), False),
-    (W.custom(1, 3, 129, 128, seed=14), True),
-    (W.custom(2, 2, 300, 64, seed=15), True),
-    (W.custom(1, 2, 1000, 128, seed=16, q_outlier_frac=1e-3), False),
-    (W.custom(1, 2, 1536, 64, "fp16", seed=17), False),
-    (W.custom(1, 2, 1100, 128, seed=18), True),
+    Case(W.SMALL),
+    Case(W.custom(1, 2, 1, 128, seed=11)),
+    Case(W.custom(1, 2, 17, 64, "fp16", seed=12), causal=True),
+    Case(W.custom(1, 3, 127, 128, seed=13)),
+    Case(W.custom(1, 3, 129, 128, seed=14), causal=True),
+    Case(W.custom(2, 2, 300, 64, seed=15), causal=True),
+    Case(W.custom(1, 2, 1000, 128, seed=16, q_outlier_frac=1e-3), miss=OUTLIERS.format("block", 0.99574)),
+    Case(W.custom(1, 2, 1536, 64, "fp16", seed=17)),
+    Case(W.custom(1, 2, 1100, 128, seed=18), causal=True),
+    Case(W.MID, rows=tuple(np.concatenate([np.arange(0, 4096, 61), [4095]]).tolist()),
+         miss=OUTLIERS.format("block", 0.99741)),
+    # the bench's workload and launch (library-owned workspace via sattn_fwd)
+    Case(W.VIDEO_32760, rows=sample_rows(32760, 60, 0, (0, 127, 32639, 32759)),
+         heads=((0, 0), (0, 5), (0, 11), (0, 7)), via_fwd=True, miss=OUTLIERS.format("block", 0.99749)),
+    Case(W.VIDEO_75600, rows=sample_rows(75600, 60, 1, (0, 75599, 75520, 75519)),
+         heads=((0, 0), (0, 13), (0, 26), (0, 39))),
+] + [Case(W.sweep(d, N, c), causal=c, rows=sample_rows(N, 48, N, (0, N - 1)), heads=((0, 0), (3, 31), (1, 17)))
+     for d, N, c in [(64, 1024, True), (128, 2048, False), (64, 8192, False), (128, 16384, True)]]
+
+# one INT8 scale per query token ("thread-level" granularity)
+QTOK_CASES = [
+    Case(W.custom(1, 2, 300, 64, "fp16", seed=51), causal=True, q_per_token=True),
+    Case(W.custom(1, 3, 129, 128, seed=52), q_per_token=True),
+    Case(W.custom(1, 2, 1000, 128, seed=16, q_outlier_frac=1e-3), q_per_token=True,
+         miss=OUTLIERS.format("token", 0.99814)),
+    Case(W.MID, rows=tuple(np.concatenate([np.arange(0, 4096, 61), [4095]]).tolist()), q_per_token=True,
+         miss=OUTLIERS.format("token", 0.99854)),
+    Case(W.VIDEO_32760, rows=sample_rows(32760, 60, 0, (0, 127, 32639, 32759)),
+         heads=((0, 0), (0, 5), (0, 11), (0, 7)), via_fwd=True, q_per_token=True,
+         miss=OUTLIERS.format("token", 0.99831)),
 ]
 
 
-@pytest.mark.parametrize("w,causal", ATTN_CASES, ids=lambda x: getattr(x, "name", str(x)))
-def test_attention_matches_oracle(w, causal):
-    _check_attention(w, causal)
+@pytest.mark.parametrize("case", ATTN_CASES + QTOK_CASES, ids=lambda c: c.id)
+def test_attention_matches_oracle(case):
+    check_parity(case, "i8f8")
 
 
-def test_mid_workload_all_heads_sampled_rows():
-    w = W.MID
-    rows = np.concatenate([np.arange(0, 4096, 61), [4095]])
-    _check_attention(w, False, rows=rows)
+@pytest.mark.parametrize("case", miss_params(ATTN_CASES + QTOK_CASES))
+def test_cosine_bar_where_the_scheme_misses_it(case):
+    check_cosine_bar(case, "i8f8")
 
 
-def test_video_32760_bench_launch_sampled():
-    """The bench's workload and launch (library-owned workspace via sattn_fwd)."""
-    w = W.VIDEO_32760
-    rows = np.concatenate([np.random.default_rng(0).choice(w.N, 60, replace=False), [0, 127, 32639, 32759]])
-    _check_attention(w, False, rows=rows, heads=[(0, 0), (0, 5), (0, 11), (0, 7)], via_fwd=True)
+def _check_attention(w, causal):
+    check_parity(Case(w, causal=causal), "i8f8")
 
 
-def test_video_75600_sampled():
-    w = W.VIDEO_75600
-    rows = np.concatenate([np.random.default_rng(1).choice(w.N, 60, replace=False), [0, 75599, 75520, 75519]])
-    _check_attention(w, False, rows=rows, heads=[(0, 0), (0, 13), (0, 26), (0, 39)])
-
-
-@pytest.mark.parametrize("d,N,causal", [(64, 1024, True), (128, 2048, False), (64, 8192, False),
-                                        (128, 16384, True)])
-def test_sweep_points_sampled(d, N, causal):
-    w = W.sweep(d, N, causal)
-    rows = np.concatenate([np.random.default_rng(N).choice(N, 48, replace=False), [0, N - 1]])
-    _check_attention(w, causal, rows=rows, heads=[(0, 0), (3, 31), (1, 17)])
+@pytest.mark.parametrize("w", [W.custom(1, 2, 300, 128, seed=53, q_outlier_frac=1e-3),
+                               W.custom(2, 1, 129, 64, "fp16", seed=54)], ids=lambda w: w.name)
+def test_per_token_q_quantizer_bit_exact(w):
+    q, k, v = W.make_inputs(w, "cuda")
+    ws = sattn.quantize(q, k, v, q_per_token=True)
+    torch.cuda.synchronize()
+    lay = sattn.workspace_layout(w.B, w.H, w.N, w.d, dtype=q.dtype, q_per_token=True)
+    h = ws.cpu().numpy()
+    BH, N, d = w.B * w.H, w.N, w.d
+    g_q = h[lay["q8"]: lay["q8"] + BH * N * d].view(np.int8).reshape(BH, N, d)
+    g_sq = h[lay["sq"]: lay["sq"] + BH * N * 4].view(np.float32).reshape(BH, N)
+    qf = _f32(q)
+    for b in range(w.B):
+        for hh in range(w.H):
+            codes, sc = Qz.quant_int8_blocks(qf[b, hh], 1)
+            assert np.array_equal(g_sq[b * w.H + hh], sc), "per-token Q scales"
+            assert np.array_equal(g_q[b * w.H + hh], codes), "per-token Q codes"
 
 
 # ------------------------------------------------------------------ degenerate inputs
@@ -196,3 +193,25 @@ def test_repeated_calls_are_deterministic():
 def test_fp16_and_bf16_agree_with_their_own_oracles():
     for dt in ("fp16", "bf16"):
         _check_attention(W.custom(1, 2, 400, 64, dt, seed=24), False)
+
+
+@pytest.mark.parametrize("what", ["q", "q_token", "k", "v"])
+def test_nan_input_spoils_the_outputs_the_oracle_says(what):
+    """NaN propagates through the max-based scales: the NaN pattern of the output
+    equals the oracle's (a Q block's rows or one token's row, the whole head, or
+    one output column) and every other element keeps parity."""
+    w = W.custom(1, 2, 300, 64, seed=72)
+    q, k, v = W.make_inputs(w, "cuda")
+    pos = {"q": (q, (0, 0, 140, 3)), "q_token": (q, (0, 0, 140, 3)), "k": (k, (0, 1, 7, 30)),
+           "v": (v, (0, 0, 250, 9))}[what]
+    pos[0][pos[1]] = float("nan")
+    qtok = what == "q_token"
+    out = sattn.fwd(q, k, v, q_per_token=qtok)
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy()[0]
+    emu = A.attn_quant_emul_i8f8(_f32(q), _f32(k), _f32(v), block_q=1 if qtok else 128,
+                                 tau=sattn.I8F8_LAZY_TAU)
+    assert np.isnan(emu).any()
+    assert np.array_equal(np.isnan(got), np.isnan(emu))
+    fin = ~np.isnan(emu)
+    assert np.abs(got[fin] - emu[fin]).max() <= 2e-2

@@ -2,9 +2,11 @@
 
 Quantiser outputs (E2M1 codes, E4M3 block scales, K mean) are compared bit for
 bit.  Attention outputs are compared element by element with the oracle's
-NVFP4 emulation: max |err| <= 6e-2 and mean |err| <= 6e-3, and with the exact
-float64 attention by cosine similarity (>= 0.995, or no worse than the
-emulation itself by 1e-3 where the scheme's own accuracy is lower).
+NVFP4 emulation: max |err| <= 6e-2 and mean |err| <= 6e-3; and with the exact
+float64 attention by cosine similarity >= 0.995.  FP4 Q and K alone cost more
+than that on these Gaussian inputs (the emulation's cosine is 0.95-0.99), so
+on every input but the trivial one the cosine test is a strict expected
+failure that records the scheme's measured value (see tests/gpu_parity.py).
 """
 
 import numpy as np
@@ -13,14 +15,12 @@ import torch
 
 import bit_quantized_attention_smooth_b200 as sattn
 from bit_quantized_attention_smooth_b200 import build as sattn_build
-from oracle import attention as A
 from oracle import quant as Qz
 from oracle.formats import e2m1_decode
 import workloads as W
+from tests.gpu_parity import Case, check_cosine_bar, check_parity, miss_params, sample_rows
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS, MEAN_ABS, COS = 6e-2, 6e-3, 0.995
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -104,67 +104,31 @@ def test_nvfp4_quantizer_bit_exact(w):
             assert np.array_equal(gsv[:, :nblk_tok], z["vt_sc_codes"][:, :nblk_tok])
 
 
-def _check(w, causal, rows=None, heads=None, via_fwd=False):
-    q, k, v = W.make_inputs(w, "cuda")
-    if via_fwd:
-        out = sattn.fwd(q, k, v, causal=causal, mode="nvfp4")
-    else:
-        ws = sattn.quantize(q, k, v, mode="nvfp4")
-        out = sattn.fwd_quantized(ws, q.shape, causal=causal, mode="nvfp4", dtype=q.dtype)
-    torch.cuda.synchronize()
-    if heads is None:
-        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    rows_idx = np.arange(w.N) if rows is None else np.asarray(rows)
-    qf, kf, vf = W.make_heads_f32(w, heads)
-    emu = A.attn_quant_emul_nvfp4(qf, kf, vf, causal=causal, rows=rows_idx)
-    exact = A.attn_exact(qf, kf, vf, causal=causal, rows=rows_idx)
-    o = out.float().cpu().numpy()
-    got = np.stack([o[b, h][rows_idx] for (b, h) in heads])
-    err = np.abs(got - emu)
-    cos_gpu, cos_emu = A.cosine(exact, got), A.cosine(exact, emu)
-    print(f"{w.name} causal={causal}: max|err|={err.max():.3e} mean|err|={err.mean():.3e} "
-          f"cos(gpu,exact)={cos_gpu:.6f} cos(emul,exact)={cos_emu:.6f}")
-    assert np.isfinite(got).all()
-    assert err.max() <= MAX_ABS
-    assert err.mean() <= MEAN_ABS
-    assert cos_gpu >= min(COS, cos_emu - 1e-3)
-
+SCHEME = "FP4 E2M1 Q/K/V/P: the scheme's own cosine to exact attention is {:.5f} here"
 
 ATTN_CASES = [
-    (W.custom(1, 2, 256, 64, "fp16", seed=41), False),
-    (W.custom(1, 2, 1, 128, seed=42), False),
-    (W.custom(1, 2, 17, 64, seed=43), True),
-    (W.custom(1, 3, 129, 128, seed=44), True),
-    (W.custom(2, 2, 300, 64, seed=45), False),
-    (W.custom(1, 2, 1000, 128, seed=46, q_outlier_frac=1e-3), False),
-    (W.custom(1, 2, 1100, 128, seed=47), True),
-]
+    Case(W.custom(1, 2, 256, 64, "fp16", seed=41), miss=SCHEME.format(0.98243)),
+    Case(W.custom(1, 2, 1, 128, seed=42)),
+    Case(W.custom(1, 2, 17, 64, seed=43), causal=True, miss=SCHEME.format(0.9893)),
+    Case(W.custom(1, 3, 129, 128, seed=44), causal=True, miss=SCHEME.format(0.98631)),
+    Case(W.custom(2, 2, 300, 64, seed=45), miss=SCHEME.format(0.98255)),
+    Case(W.custom(1, 2, 1000, 128, seed=46, q_outlier_frac=1e-3), miss=SCHEME.format(0.96535)),
+    Case(W.custom(1, 2, 1100, 128, seed=47), causal=True, miss=SCHEME.format(0.98548)),
+    Case(W.MID, rows=tuple(np.concatenate([np.arange(0, 4096, 97), [4095]]).tolist()), miss=SCHEME.format(0.9628)),
+    Case(W.VIDEO_32760, rows=sample_rows(32760, 40, 2, (0, 32759)), heads=((0, 0), (0, 6), (0, 11)), via_fwd=True,
+         miss=SCHEME.format(0.94162)),
+    Case(W.VIDEO_75600, rows=sample_rows(75600, 40, 3, (0, 75599)), heads=((0, 0), (0, 21), (0, 39)),
+         miss=SCHEME.format(0.9817)),
+] + [Case(W.sweep(d, N, c), causal=c, rows=sample_rows(N, 32, N + 1, (0, N - 1)), heads=((0, 0), (3, 31)),
+          miss=SCHEME.format(cos))
+     for d, N, c, cos in [(64, 2048, True, 0.99340), (128, 8192, False, 0.98098)]]
 
 
-@pytest.mark.parametrize("w,causal", ATTN_CASES, ids=lambda x: getattr(x, "name", str(x)))
-def test_nvfp4_attention_matches_oracle(w, causal):
-    _check(w, causal)
+@pytest.mark.parametrize("case", ATTN_CASES, ids=lambda c: c.id)
+def test_nvfp4_attention_matches_oracle(case):
+    check_parity(case, "nvfp4")
 
 
-def test_nvfp4_mid_workload_sampled():
-    rows = np.concatenate([np.arange(0, 4096, 97), [4095]])
-    _check(W.MID, False, rows=rows)
-
-
-def test_nvfp4_video_32760_sampled():
-    w = W.VIDEO_32760
-    rows = np.concatenate([np.random.default_rng(2).choice(w.N, 40, replace=False), [0, 32759]])
-    _check(w, False, rows=rows, heads=[(0, 0), (0, 6), (0, 11)], via_fwd=True)
-
-
-def test_nvfp4_video_75600_sampled():
-    w = W.VIDEO_75600
-    rows = np.concatenate([np.random.default_rng(3).choice(w.N, 40, replace=False), [0, 75599]])
-    _check(w, False, rows=rows, heads=[(0, 0), (0, 21), (0, 39)])
-
-
-@pytest.mark.parametrize("d,N,causal", [(64, 2048, True), (128, 8192, False)])
-def test_nvfp4_sweep_points_sampled(d, N, causal):
-    w = W.sweep(d, N, causal)
-    rows = np.concatenate([np.random.default_rng(N + 1).choice(N, 32, replace=False), [0, N - 1]])
-    _check(w, causal, rows=rows, heads=[(0, 0), (3, 31)])
+@pytest.mark.parametrize("case", miss_params(ATTN_CASES))
+def test_nvfp4_cosine_bar_where_the_scheme_misses_it(case):
+    check_cosine_bar(case, "nvfp4")
