@@ -8,8 +8,11 @@ starts; L2 is flushed (a 256 MiB write) between steps, outside the per-step
 events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--mode i8f8|nvfp4] [--workload NAME] [--causal] [--q-per-token]
+    python bench.py --sweep [--steps K]      # the B=4 H=32 sweep, both modes
 
-Prints ONE JSON line on rank 0.  Under torchrun (N > 1) every rank runs its own
+Prints ONE JSON line on rank 0 (the sweep: one per point and mode).  Step and
+kernel times are medians over the timed steps.  Under torchrun (N > 1) every rank runs its own
 copy of the workload (independent heads: no data exchange), the step time is
 the max over ranks and ``value`` counts the operations of all ranks.
 ``--impl reference`` times the CPU oracle instead (rank 0 only), each step a
@@ -18,6 +21,7 @@ bounded sample of the same workload.
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -127,23 +131,26 @@ def oracle_sample(w, target_s, rows_n=None):
 
     Returns (ops processed, seconds, rows).  Quantisation of the whole head is
     part of every sample (the oracle always quantises full heads)."""
+    import functools
     from oracle import attention as A
+    from bit_quantized_attention_smooth_b200 import I8F8_LAZY_TAU
+    emul = functools.partial(A.attn_quant_emul_i8f8, tau=I8F8_LAZY_TAU)
     qf, kf, vf = W.make_heads_f32(w, [(0, 0)])
     if rows_n is not None:
         rows = np.linspace(0, w.N - 1, rows_n).astype(np.int64)
         t0 = time.perf_counter()
-        A.attn_quant_emul_i8f8(qf, kf, vf, rows=rows)
+        emul(qf, kf, vf, rows=rows)
         return 4.0 * rows_n * w.N * w.d, time.perf_counter() - t0, rows_n
-    A.attn_quant_emul_i8f8(qf, kf, vf, rows=np.arange(1))            # warm caches
+    emul(qf, kf, vf, rows=np.arange(1))            # warm caches
     t0 = time.perf_counter()
-    A.attn_quant_emul_i8f8(qf, kf, vf, rows=np.arange(65))
+    emul(qf, kf, vf, rows=np.arange(65))
     t65 = time.perf_counter() - t0
     # linear through the origin: over-estimates the per-row cost (the time
     # includes the head's quantisation), so the sample stays within target_s
     rows_n = int(max(1, min(w.N, 65 * target_s / t65)))
     rows = np.linspace(0, w.N - 1, rows_n).astype(np.int64)
     t0 = time.perf_counter()
-    A.attn_quant_emul_i8f8(qf, kf, vf, rows=rows)
+    emul(qf, kf, vf, rows=rows)
     dt = time.perf_counter() - t0
     return 4.0 * rows_n * w.N * w.d, dt, rows_n
 
@@ -192,8 +199,92 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------- GPU arm
 
-def run_gpu(args):
-    import bit_quantized_attention_smooth_b200 as sattn
+PEAK_RATIO = {"i8f8": 2.0, "nvfp4": 4.0}       # dense INT8/FP8 = 2 x bf16, FP4 = 4 x bf16 (nominal)
+DATASHEET = {"i8f8": 4500.0, "nvfp4": 9000.0}  # dense TOPS
+
+
+def median(xs):
+    return statistics.median(xs) if xs else float("nan")
+
+
+class ModeRunner:
+    """One mode on one set of device inputs: its workspace, device-timed steps
+    (quantize + attention, L2 flushed before each) and an accuracy sample."""
+
+    def __init__(self, sattn, q, k, v, causal, mode, q_per_token, flush):
+        self.sattn, self.q, self.k, self.v = sattn, q, k, v
+        self.causal, self.mode, self.qtok, self.flush = causal, mode, q_per_token, flush
+        B, H, N, d = q.shape
+        self.shape = (B, H, N, d)
+        self.ws = torch.empty(sattn.workspace_bytes(B, H, N, d, mode=mode, dtype=q.dtype, q_per_token=q_per_token),
+                              dtype=torch.uint8, device=q.device)
+        self.out = torch.empty_like(q)
+
+    def step(self, stream):
+        s = self.sattn
+        s.quantize(self.q, self.k, self.v, mode=self.mode, workspace=self.ws, q_per_token=self.qtok)
+        mid = torch.cuda.Event(enable_timing=True)
+        mid.record(stream)
+        s.fwd_quantized(self.ws, self.shape, causal=self.causal, mode=self.mode, dtype=self.q.dtype, out=self.out,
+                        q_per_token=self.qtok)
+        return mid
+
+    def timed(self, n, stream):
+        """n steps; returns lists of (step ms, attention ms, quantize ms)."""
+        evs = []
+        for _ in range(n):
+            self.flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e2 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            e1 = self.step(stream)
+            e2.record(stream)
+            evs.append((e0, e1, e2))
+        torch.cuda.synchronize()
+        return ([a.elapsed_time(c) for a, b, c in evs], [b.elapsed_time(c) for a, b, c in evs],
+                [a.elapsed_time(b) for a, b, c in evs])
+
+    def warm(self, n, stream):
+        for _ in range(n):
+            self.flush.zero_()
+            self.step(stream)
+        torch.cuda.synchronize()
+
+    def cosine_to_exact(self, heads, rows):
+        """Cosine similarity of the output rows to exact float64 attention of the
+        same device inputs (plain torch on the GPU), over the sampled heads x rows."""
+        got, ref = [], []
+        idx = torch.as_tensor(rows, device=self.q.device)
+        B, H, N, d = self.shape
+        scale = 1.0 / math.sqrt(d)
+        for (b, h) in heads:
+            qh = self.q[b, h].double()[idx]
+            S = (qh @ self.k[b, h].double().T) * scale
+            if self.causal:
+                S = S.masked_fill(torch.arange(N, device=S.device)[None, :] > idx[:, None], float("-inf"))
+            ref.append(torch.softmax(S, dim=1) @ self.v[b, h].double())
+            got.append(self.out[b, h].double()[idx])
+        a, b_ = torch.cat(got).flatten(), torch.cat(ref).flatten()
+        return float(a @ b_ / (a.norm() * b_.norm()))
+
+
+def accuracy_sample(w, n_rows=64, n_heads=2):
+    heads = [(0, 0), (w.B - 1, w.H - 1)][:n_heads]
+    rows = np.unique(np.linspace(0, w.N - 1, n_rows).astype(np.int64))
+    return heads, rows
+
+
+def attention_report(w, mode, causal, attn_ms, peaks):
+    ops = w.ops()
+    tops = ops / (attn_ms * 1e-3) / 1e12
+    r = {"ms": attn_ms, "tops": tops, "frac_of_datasheet": tops / DATASHEET[mode],
+         "frac_of_measured_peak": tops / (PEAK_RATIO[mode] * peaks["bf16_tflops"])}
+    if causal:
+        r["tops_causal_half_count"] = tops / 2     # the algorithmic work of a causal pass is half the pairs
+    return r
+
+
+def init_dist():
     ws_n, rank, local = dist_env()
     if ws_n > 1:
         import datetime
@@ -203,50 +294,69 @@ def run_gpu(args):
                                 device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
+    return ws_n, rank, local
+
+
+def run_sweep(args):
+    """The B=4, H=32 sweep (d in {64,128}, N in 1024..32768, causal and
+    non-causal), both modes: one JSON line per point and mode.  Inputs follow
+    the workload recipe but are drawn on the device (a different random stream
+    from the CPU recipe the parity tests use), so that 1 GB tensors are made
+    in milliseconds."""
+    import bit_quantized_attention_smooth_b200 as sattn
+    ws_n, rank, _ = init_dist()
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = WORKLOAD
+    peaks, _ = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for (d, N, causal) in W.SWEEP_POINTS:
+        w = W.sweep(d, N, causal)
+        q, k, v = W.make_inputs_device(w, dev)
+        for mode in ("i8f8", "nvfp4"):
+            r = ModeRunner(sattn, q, k, v, causal, mode, False, flush)
+            r.warm(args.warmup, stream)
+            step_ms, attn_ms, quant_ms = r.timed(args.steps, stream)
+            step_med, attn_med = max_over_ranks([median(step_ms), median(attn_ms)], dev)
+            heads, rows = accuracy_sample(w, 32, 2)
+            cos = r.cosine_to_exact(heads, rows)
+            if rank == 0:
+                print(json.dumps({"sweep": True, "workload": w.name, "mode": mode, "B": w.B, "H": w.H, "N": N, "d": d,
+                                  "causal": causal, "steps": args.steps, "ms_per_step": step_med,
+                                  "value": job_throughput(w.ops(), ws_n, step_med), "unit": "TOPS",
+                                  "quantize_ms": median(quant_ms),
+                                  "attention_kernel": attention_report(w, mode, causal, attn_med, peaks),
+                                  "cos_vs_exact": cos, "accuracy_sample": f"{len(heads)} heads x {len(rows)} rows",
+                                  "inputs": "device-drawn (same recipe, other random stream)"}), flush=True)
+            del r
+        del q, k, v
+        torch.cuda.empty_cache()
+    if ws_n > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_gpu(args):
+    import bit_quantized_attention_smooth_b200 as sattn
+    ws_n, rank, local = init_dist()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.WORKLOADS[args.workload]
+    causal = bool(args.causal)
     q, k, v = W.make_inputs(w, dev)
     B, H, N, d = q.shape
     ops = w.ops()
     mode = args.mode
-    workspace = torch.empty(sattn.workspace_bytes(B, H, N, d, mode=mode), dtype=torch.uint8, device=dev)
-    out = torch.empty_like(q)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    def step(m=mode, ws=workspace):
-        sattn.quantize(q, k, v, mode=m, workspace=ws)
-        ev_mid = torch.cuda.Event(enable_timing=True)
-        ev_mid.record(stream)
-        sattn.fwd_quantized(ws, (B, H, N, d), mode=m, dtype=q.dtype, out=out)
-        return ev_mid
-
-    def timed_steps(n, m=mode, ws=workspace):
-        """n device-timed steps with an L2 flush before each; returns (step ms list, attention ms list)."""
-        evs = []
-        for _ in range(n):
-            flush.zero_()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e2 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            e1 = step(m, ws)
-            e2.record(stream)
-            evs.append((e0, e1, e2))
-        torch.cuda.synchronize()
-        return [a.elapsed_time(c) for a, b, c in evs], [b.elapsed_time(c) for a, b, c in evs], \
-            [a.elapsed_time(b) for a, b, c in evs]
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
+    main = ModeRunner(sattn, q, k, v, causal, mode, args.q_per_token, flush)
+    main.warm(args.warmup, stream)
     if args.profile:
         # Profiling mode (for ncu): the same steps, no e2e leg, no CPU baseline.
         for _ in range(args.steps):
             flush.zero_()
-            step()
+            main.step(stream)
         torch.cuda.synchronize()
-        print(json.dumps({"profile": True, "workload": w.name, "steps": args.steps,
+        print(json.dumps({"profile": True, "workload": w.name, "mode": mode, "steps": args.steps,
                           "device_error_word": sattn.device_error()}), flush=True)
         return 0
 
@@ -259,19 +369,28 @@ def run_gpu(args):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    step_ms, attn_ms, quant_ms = timed_steps(args.steps)
+    sattn.kernel_launches(reset=True)
+    step_ms, attn_ms, quant_ms = main.timed(args.steps, stream)
+    launches = sattn.kernel_launches()
     barrier()
     clocks = sampler.stop()
-    # the other mode on the same inputs (reported beside the headline mode)
-    other = "nvfp4" if mode == "i8f8" else "i8f8"
-    ws_other = torch.empty(sattn.workspace_bytes(B, H, N, d, mode=other), dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        step(other, ws_other)
-    o_step, o_attn, o_quant = timed_steps(args.steps, other, ws_other)
-    del ws_other
-    ms = sum(step_ms) / len(step_ms)
-    attn_avg = sum(attn_ms) / len(attn_ms)
-    ms, attn_avg = max_over_ranks([ms, attn_avg], dev)
+    ms, attn_med = max_over_ranks([median(step_ms), median(attn_ms)], dev)
+    heads, rows = accuracy_sample(w)
+    cos_main = main.cosine_to_exact(heads, rows)
+
+    # the other mode on the same inputs, and per-token Q scales (I8QK_F8PV), beside the headline
+    legs = {}
+    for name, (m, qtok) in {"nvfp4": ("nvfp4", False), "i8f8": ("i8f8", False),
+                            "i8f8_q_per_token": ("i8f8", True)}.items():
+        if m == mode and qtok == args.q_per_token:
+            continue
+        r = ModeRunner(sattn, q, k, v, causal, m, qtok, flush)
+        r.warm(args.warmup, stream)
+        o_step, o_attn, o_quant = r.timed(args.steps, stream)
+        legs[name] = {"ms_per_step": median(o_step), "quantize_ms": median(o_quant),
+                      "value": ops / (median(o_step) * 1e-3) / 1e12,
+                      "attention_kernel_ms": median(o_attn), "cos_vs_exact": r.cosine_to_exact(heads, rows)}
+        del r
 
     # ---- end to end through the C-ABI call on host buffers (pinned): every
     # step copies q, k, v in and the output back, pipelined by the library in
@@ -280,7 +399,7 @@ def run_gpu(args):
     hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
 
     def e2e_step():
-        sattn.fwd_host(hq, hk, hv, out=hout, mode=mode)
+        sattn.fwd_host(hq, hk, hv, out=hout, causal=causal, mode=mode, q_per_token=args.q_per_token)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
@@ -299,23 +418,18 @@ def run_gpu(args):
     line = None
     if rank == 0:
         peaks, src = measured_peaks()
-        ratio = {"i8f8": 2.0, "nvfp4": 4.0}               # dense INT8/FP8 = 2 x bf16, FP4 = 4 x bf16 (nominal)
-        datasheet = {"i8f8": 4500.0, "nvfp4": 9000.0}
-        peak_i8 = ratio[mode] * peaks["bf16_tflops"]
-        achieved = ops / (attn_avg * 1e-3) / 1e12
-        o_ms, o_attn_avg = sum(o_step) / len(o_step), sum(o_attn) / len(o_attn)
-        o_achieved = ops / (o_attn_avg * 1e-3) / 1e12
-        other_line = {"mode": other, "value": ops / (o_ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": o_ms,
-                      "attention_kernel": {"ms": o_attn_avg, "tops": o_achieved,
-                                           "frac_of_datasheet": o_achieved / datasheet[other],
-                                           "frac_of_measured_peak": o_achieved / (ratio[other] * peaks["bf16_tflops"])},
-                      "quantize_ms": sum(o_quant) / len(o_quant)}
+        peak = PEAK_RATIO[mode] * peaks["bf16_tflops"]
+        att = attention_report(w, mode, causal, attn_med, peaks)
+        achieved = att["tops"]
+        for name, leg in legs.items():
+            m = "nvfp4" if name == "nvfp4" else "i8f8"
+            leg["attention_kernel"] = attention_report(w, m, causal, leg.pop("attention_kernel_ms"), peaks)
         traffic = None
-        tpath = os.path.join(ROOT, "profiles", "attn_i8f8_traffic.json")
+        tpath = os.path.join(ROOT, "profiles", f"attn_{mode}_traffic.json")
         if os.path.exists(tpath):
             with open(tpath) as f:
                 tj = json.load(f)
-            if tj.get("kernel_hash") == kernel_hash():
+            if tj.get("kernel_hash") == kernel_hash(mode) and tj.get("workload") == w.name:
                 traffic = tj.get("dram_bytes_per_launch_full")
         cpu = None
         if ws_n == 1 and not args.no_cpu_baseline:
@@ -326,9 +440,9 @@ def run_gpu(args):
         value = job_throughput(ops, ws_n, ms)
         try:                       # a reported second bound; never lose the bench line over it
             sm_mhz = clocks["sm_mhz"] if clocks and clocks.get("sm_mhz") else 1965.0
-            mufu = mufu_bound(float(w.B) * w.H * w.N * w.N, attn_avg,
-                              torch.cuda.get_device_properties(dev).multi_processor_count, sm_mhz)
-            mufu["binds"] = mufu["frac"] > achieved / peak_i8      # the bound this kernel is closer to
+            pairs = float(w.B) * w.H * w.N * w.N / (2 if causal else 1)
+            mufu = mufu_bound(pairs, attn_med, torch.cuda.get_device_properties(dev).multi_processor_count, sm_mhz)
+            mufu["binds"] = mufu["frac"] > achieved / peak      # the bound this kernel is closer to
         except Exception as exc:   # noqa: BLE001
             mufu = {"bound": "mufu", "error": repr(exc)}
         line = {
@@ -339,23 +453,27 @@ def run_gpu(args):
                       else "nvfp4 QK^T / nvfp4 PV (e2m1 + e4m3 block scales; fp32 softmax + accumulation)"),
             "data": "synthetic",
             "config": {"workload": w.name, "mode": "I8QK_F8PV" if mode == "i8f8" else "NVFP4", "B": w.B, "H": w.H,
-                       "N": w.N, "d": w.d,
-                       "causal": False, "io_dtype": w.dtype, "parallelism": f"replicas x{ws_n} (independent heads)",
+                       "N": w.N, "d": w.d, "causal": causal, "io_dtype": w.dtype,
+                       "q_scales": "per token" if args.q_per_token else "per 128-token block",
+                       "lazy_max_tau": sattn.I8F8_LAZY_TAU if mode == "i8f8" else None,
+                       "parallelism": f"replicas x{ws_n} (independent heads)",
                        "l2": "flushed between steps (256 MiB write, outside the step events)"},
-            "attention_kernel": {"ms": attn_avg, "tops": achieved,
-                                 "frac_of_datasheet": achieved / datasheet[mode]},
-            "other_mode": other_line,
-            "quantize_ms": sum(quant_ms) / len(quant_ms),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_i8, "unit": "TFLOP/s",
-                         "frac": achieved / peak_i8, "traffic": traffic,
-                         "peak_source": f"{src}: {ratio[mode]:.0f} x bf16 burst {peaks['bf16_tflops']} "
+            "attention_kernel": att,
+            "quantize_ms": median(quant_ms),
+            "timing": "median of the timed steps (CUDA events on the launching stream); max over ranks",
+            "accuracy": {"cos_vs_exact": cos_main, "sample": f"{len(heads)} heads x {len(rows)} rows, "
+                                                             "exact float64 attention of the same device inputs"},
+            "other_legs": legs,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{src}: {PEAK_RATIO[mode]:.0f} x bf16 burst {peaks['bf16_tflops']} "
                                         f"(nominal dense ratio of {mode} to bf16)"},
             "roofline_mufu": mufu,
             "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(ops, ws_n, e2e_ms), "unit": "TOPS",
                     "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
-                    "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e2e_ms},
-            "gpu_launches": 5 * args.steps,   # per step: stats, quant Q, quant K, quant V, attention
+                    "d2h_bytes_per_step": q.numel() * q.element_size(), "ms_per_step": e2e_ms},
+            "gpu_launches": launches,
             "clocks": clocks,
             "device_error_word": err,
         }
@@ -367,10 +485,10 @@ def run_gpu(args):
     return 0
 
 
-def kernel_hash():
+def kernel_hash(mode="i8f8"):
     import hashlib
     h = hashlib.sha256()
-    for f in ("attn_i8f8.cuh", "ptx.cuh"):
+    for f in (f"attn_{mode}.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "bit_quantized_attention_smooth_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -385,6 +503,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="i8f8", choices=["i8f8", "nvfp4"])
+    ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--causal", action="store_true")
+    ap.add_argument("--q-per-token", action="store_true", help="I8QK_F8PV with one Q scale per token")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the B=4 H=32 sweep in both modes (one JSON line per point and mode)")
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps of the GPU path only (for ncu captures)")
     args = ap.parse_args()
@@ -392,6 +515,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_gpu(args)
 
 

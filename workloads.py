@@ -118,3 +118,20 @@ def custom(B, H, N, d, dtype="bf16", causal=False, seed=0, q_outlier_frac=0.0):
     """Workload of arbitrary shape with the same recipe (tests: ragged, edge cases)."""
     return Workload(f"custom-B{B}H{H}N{N}d{d}", B, H, N, d, dtype, causal=causal, seed=seed,
                     q_outlier_frac=q_outlier_frac)
+
+
+def make_inputs_device(w: Workload, device):
+    """The same distributions as ``make_inputs``, drawn on ``device`` with one
+    device generator seeded by the workload seed (a different random stream:
+    for timing large workloads, not for comparison with the CPU oracle)."""
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    shape = (w.B, w.H, w.N, w.d)
+    q = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    k += torch.randn((w.B, w.H, 1, w.d), generator=g, device=device, dtype=torch.float32) * 3.0
+    v = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if w.q_outlier_frac > 0:
+        mask = torch.rand(shape, generator=g, device=device, dtype=torch.float32) < w.q_outlier_frac
+        q = torch.where(mask, q * w.q_outlier_mult, q)
+    dt = w.torch_dtype
+    return q.to(dt), k.to(dt), v.to(dt)
