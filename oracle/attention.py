@@ -53,17 +53,42 @@ def _sel(B, H, N, heads, rows):
     return heads, rows
 
 
-def _valid_mask(rows, cols, n, causal):
-    """Key j is valid for query i iff j < N and (not causal or j <= i)."""
+BLOCK = 128   # query and key block of the block-sparse mask
+
+
+def _valid_mask(rows, cols, n, causal, blocks=None):
+    """Key j is valid for query i iff j < N and (not causal or j <= i) and, with
+    a block-sparse mask ``blocks`` [nblk, nblk] of one head, the 128 x 128 block
+    (i // 128, j // 128) is kept (nonzero)."""
     m = np.broadcast_to(cols[None, :] < n, (len(rows), len(cols))).copy()
     if causal:
         m &= cols[None, :] <= rows[:, None]
+    if blocks is not None:
+        m &= np.asarray(blocks, dtype=bool)[rows // BLOCK][:, cols // BLOCK]
     return m
 
 
-def attn_exact(q, k, v, causal=False, sm_scale=None, heads=None, rows=None):
+def _head_blocks(block_mask, b, h):
+    return None if block_mask is None else block_mask[b, h]
+
+
+def _safe_div(acc, l):
+    """acc / l per row; a row with no valid key (every block of its query block
+    skipped) has l = 0 and is defined as zeros."""
+    l = np.asarray(l, dtype=np.float64)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = acc / l[:, None]
+    return np.where(l[:, None] == 0, 0.0, out)
+
+
+def attn_exact(q, k, v, causal=False, sm_scale=None, heads=None, rows=None, block_mask=None):
     """O = softmax(Q K^T * sm_scale [masked]) V in float64.
 
+    ``block_mask`` [B, H, nblk, nblk] (nblk = ceil(N / 128)), optional: keys of
+    a skipped 128 x 128 block are left out of the softmax of that block's
+    queries, as if masked (the "skip" part of Sparse-Linear Attention in the
+    TurboDiffusion explainer, SLA section, with a given mask); a row whose
+    query block skips every key block is zeros.
     Returns [len(heads), len(rows), d] float64.
     """
     B, H, N, d = q.shape
@@ -74,10 +99,11 @@ def attn_exact(q, k, v, causal=False, sm_scale=None, heads=None, rows=None):
     for t, (b, h) in enumerate(heads):
         qh = q[b, h].astype(np.float64)[rows]
         S = (qh @ k[b, h].astype(np.float64).T) * s
-        S = np.where(_valid_mask(rows, cols, N, causal), S, -np.inf)
-        S = S - S.max(axis=1, keepdims=True)
-        P = np.exp(S)
-        out[t] = (P @ v[b, h].astype(np.float64)) / P.sum(axis=1, keepdims=True)
+        valid = _valid_mask(rows, cols, N, causal, _head_blocks(block_mask, b, h))
+        S = np.where(valid, S, -np.inf)
+        mx = S.max(axis=1, keepdims=True)
+        P = np.exp(S - np.where(np.isneginf(mx), 0.0, mx))
+        out[t] = _safe_div(P @ v[b, h].astype(np.float64), P.sum(axis=1))
     return out
 
 
@@ -113,7 +139,7 @@ def _online_softmax(S2, valid, tile, p_quant, pv, tau=0.0):
 
 
 def attn_online_unquantised(q, k, v, causal=False, sm_scale=None, heads=None,
-                            rows=None, block_kv=128, tau=0.0):
+                            rows=None, block_kv=128, tau=0.0, block_mask=None):
     """The same tiled online softmax with every quantiser replaced by identity.
 
     Equal to ``attn_exact`` up to float64 rounding for any ``tau`` (the
@@ -128,10 +154,10 @@ def attn_online_unquantised(q, k, v, causal=False, sm_scale=None, heads=None,
         vh = v[b, h].astype(np.float64)
         S2 = (q[b, h].astype(np.float64)[rows] @ k[b, h].astype(np.float64).T) * (s * LOG2E)
         acc, l = _online_softmax(
-            S2, _valid_mask(rows, cols, N, causal), block_kv,
+            S2, _valid_mask(rows, cols, N, causal, _head_blocks(block_mask, b, h)), block_kv,
             lambda P: (P, np.ones(P.shape[0])),
             lambda Pq, j0, j1: Pq @ vh[j0:j1], tau)
-        out[t] = acc / l[:, None]
+        out[t] = _safe_div(acc, l)
     return out
 
 
@@ -146,7 +172,7 @@ def int8_scores(qh, kh):
 
 
 def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
-                         block_q=128, block_kv=128, tau=0.0):
+                         block_q=128, block_kv=128, tau=0.0, block_mask=None):
     """INT8 QK^T / FP8 PV emulation (the I8QK_F8PV mode).
 
     Steps (TurboDiffusion explainer, section 1: QK in INT8, PV in FP8, outlier
@@ -177,10 +203,10 @@ def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=
         S2 = Sint * sq_rows[:, None] * sk_cols[None, :] * (s * LOG2E)
         c_p = P_SCALE_FP8 * 2.0 ** -tau
         acc, l = _online_softmax(
-            S2, _valid_mask(rows, cols, N, causal), block_kv,
+            S2, _valid_mask(rows, cols, N, causal, _head_blocks(block_mask, b, h)), block_kv,
             lambda P: (e4m3_round(c_p * P), np.ones(P.shape[0])),
             lambda Pq, j0, j1: Pq @ v8[j0:j1], tau)
-        out[t] = acc * z["sv"].astype(np.float64)[None, :] / (c_p * l[:, None])
+        out[t] = _safe_div(acc * z["sv"].astype(np.float64)[None, :] / c_p, l)
     return out
 
 
@@ -203,7 +229,7 @@ def two_stage_p_nvfp4(P, fmt="nvfp4"):
 
 
 def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
-                          block_kv=128, fmt="nvfp4"):
+                          block_kv=128, fmt="nvfp4", block_mask=None):
     """NVFP4 microscaled emulation (the NVFP4 mode).
 
       Q^, K'^ : NVFP4 along channels;  V^ : NVFP4 along tokens
@@ -234,10 +260,10 @@ def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows
             vv = fp4_rows(np.ascontiguousarray(v[b, h].T), fmt)[:, :N].T
         S2 = (qv[rows] @ kv.T) * (s * LOG2E)
         acc, l = _online_softmax(
-            S2, _valid_mask(rows, cols, N, causal), block_kv,
+            S2, _valid_mask(rows, cols, N, causal, _head_blocks(block_mask, b, h)), block_kv,
             lambda P: two_stage_p_nvfp4(P, fmt),
             lambda Pq, j0, j1: Pq @ vv[j0:j1])
-        out[t] = acc / l[:, None]
+        out[t] = _safe_div(acc, l)
     return out
 
 
