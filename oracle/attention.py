@@ -210,6 +210,62 @@ def attn_quant_emul_i8f8(q, k, v, causal=False, sm_scale=None, heads=None, rows=
     return out
 
 
+def attn_quant_emul_i8f8_smooth(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
+                                block_q=128, block_kv=128, smooth_q=True, p_per_token=False):
+    """The I8QK_F8PV scheme with the two variants of the SageAttention pages
+    that the kernels do not implement (tag page, SageAttention3 summary,
+    8-bit bullet [17]: per-token P; TurboDiffusion explainer, section 1:
+    outlier smoothing, here applied to Q as well as K):
+
+    * Q smoothing: qbar[b] = per-channel mean of Q over the tokens of query
+      block b (float64 sum / block length, rounded to float32);
+      Q' = Q - qbar (one float32 subtraction) is INT8-quantised per block, and
+      the correction qbar[b] . K'_j, the same for every query of block b, is
+      added to the scores in float64:
+        S2[i,j] = (q8'_i . k8_j) s_q s_k * c  +  (qbar[blk(i)] . K'_j) * c
+      With exact arithmetic Q' K'^T + qbar K'^T = Q K'^T, so the softmax is
+      unchanged.
+    * Per-token P: per row and key tile, P~ is scaled so its tile maximum maps
+      to 448, p8 = E4M3(448 P~ / r), r = rowmax_tile(P~), and the tile's
+      contribution is multiplied back by r / 448.
+    Exact (running) reference max; everything after the codes in float64.
+    """
+    from .quant import k_channel_mean, smooth_k, quant_int8_blocks, quant_v_fp8
+    B, H, N, d = q.shape
+    s = default_scale(d, sm_scale)
+    heads, rows = _sel(B, H, N, heads, rows)
+    out = np.empty((len(heads), len(rows), d))
+    cols = np.arange(N)
+    for t, (b, h) in enumerate(heads):
+        kp = smooth_k(k[b, h], k_channel_mean(k[b, h]))
+        qh = q[b, h].astype(np.float32)
+        qbar = np.zeros((N, d), dtype=np.float32)
+        if smooth_q:
+            for b0 in range(0, N, block_q):
+                blk = qh[b0:b0 + block_q]
+                qbar[b0:b0 + block_q] = (blk.astype(np.float64).sum(axis=0) / blk.shape[0]).astype(np.float32)[None, :]
+        qs = (qh - qbar).astype(np.float32)
+        q8, sq = quant_int8_blocks(qs, block_q)
+        k8, sk = quant_int8_blocks(kp, block_kv)
+        v8c, sv = quant_v_fp8(v[b, h])
+        v8 = e4m3_decode(v8c)
+        Sint = int8_scores(q8[rows], k8).astype(np.float64)
+        S2 = Sint * sq[rows // block_q].astype(np.float64)[:, None] * sk[cols // block_kv].astype(np.float64)[None, :]
+        S2 = (S2 + qbar[rows].astype(np.float64) @ kp.astype(np.float64).T) * (s * LOG2E)
+
+        def pq(P):
+            if not p_per_token:
+                return e4m3_round(P_SCALE_FP8 * P), np.ones(P.shape[0])
+            r = P.max(axis=1)
+            r = np.where(r > 0, r, 1.0)
+            return e4m3_round(P_SCALE_FP8 * P / r[:, None]), r
+
+        acc, l = _online_softmax(S2, _valid_mask(rows, cols, N, causal), block_kv, pq,
+                                 lambda Pq, j0, j1: Pq @ v8[j0:j1])
+        out[t] = _safe_div(acc * sv.astype(np.float64)[None, :] / P_SCALE_FP8, l)
+    return out
+
+
 def two_stage_p_nvfp4(P, fmt="nvfp4"):
     """Two-stage quantisation of one P~ tile [R, T] (T <= 128 keys).
 
@@ -229,7 +285,7 @@ def two_stage_p_nvfp4(P, fmt="nvfp4"):
 
 
 def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows=None,
-                          block_kv=128, fmt="nvfp4", block_mask=None):
+                          block_kv=128, fmt="nvfp4", block_mask=None, smooth_q=False):
     """NVFP4 microscaled emulation (the NVFP4 mode).
 
       Q^, K'^ : NVFP4 along channels;  V^ : NVFP4 along tokens
@@ -240,6 +296,9 @@ def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows
     ``fmt`` = "mxfp4" runs the same scheme with every FP4 operand in MXFP4
     (1 x 32 blocks, E8M0 scales): the ablation that the tag page's
     SageAttention3 summary, FP4 bullet [15], reports NVFP4 winning.
+    ``smooth_q``: Q smoothing as in ``attn_quant_emul_i8f8_smooth`` (the block
+    mean of Q is subtracted before the FP4 quantisation and qbar . K'_j is
+    added back to the scores in float64).
     """
     B, H, N, d = q.shape
     s = default_scale(d, sm_scale)
@@ -258,7 +317,18 @@ def attn_quant_emul_nvfp4(q, k, v, causal=False, sm_scale=None, heads=None, rows
             qv = fp4_rows(q[b, h], fmt)[:, :d]
             kv = fp4_rows(kp, fmt)[:, :d]
             vv = fp4_rows(np.ascontiguousarray(v[b, h].T), fmt)[:, :N].T
-        S2 = (qv[rows] @ kv.T) * (s * LOG2E)
+        if smooth_q:
+            from .quant import k_channel_mean, smooth_k
+            qh = q[b, h].astype(np.float32)
+            qbar = np.zeros_like(qh)
+            for b0 in range(0, N, 128):
+                blk = qh[b0:b0 + 128]
+                qbar[b0:b0 + 128] = (blk.astype(np.float64).sum(axis=0) / blk.shape[0]).astype(np.float32)[None, :]
+            qv = fp4_rows((qh - qbar).astype(np.float32), fmt)[:, :d]
+            kp = smooth_k(k[b, h], k_channel_mean(k[b, h])).astype(np.float64)
+            S2 = (qv[rows] @ kv.T + qbar[rows].astype(np.float64) @ kp.T) * (s * LOG2E)
+        else:
+            S2 = (qv[rows] @ kv.T) * (s * LOG2E)
         acc, l = _online_softmax(
             S2, _valid_mask(rows, cols, N, causal, _head_blocks(block_mask, b, h)), block_kv,
             lambda P: two_stage_p_nvfp4(P, fmt),
