@@ -17,7 +17,13 @@ What it computes
   Quantiser arithmetic is float32 exactly as the device performs it; everything
   after the codes is float64.
 * ``attention.attn_quant_emul_nvfp4`` -- the NVFP4 microscaled scheme with the
-  two-stage P scale.
+  two-stage P scale (``fmt="mxfp4"``: the MXFP4 ablation).
+* ``attention.attn_quant_emul_i8f8_smooth`` -- the I8F8 scheme with Q smoothing
+  and per-token P (variants the kernels do not implement).
+* ``backward.attn_fwd_bwd_8bit`` -- the 8-bit attention backward (SageBwd),
+  oracle only.
+Every attention function takes an optional block-sparse mask of 128 x 128
+(query, key) blocks to skip.
 
 Sources: the SageAttention tag page (reportify.cn), SageAttention3 summary
 (FP4-quantization bullets [15][16], 8-bit training bullet [17]); the
@@ -31,4 +37,4 @@ Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 inputs, smoothing invariance).  No function is "parity unpinned".
 """
 
-from . import formats, quant, attention  # noqa: F401
+from . import formats, quant, attention, backward  # noqa: F401
