@@ -30,7 +30,8 @@ STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
 # Every entry point declared in include/sattn.h.
 EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
            "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc",
-           "sattn_fwd_host", "sattn_kernel_launches", "sattn_debug_set_wait_limit")
+           "sattn_fwd_host", "sattn_kernel_launches", "sattn_debug_set_wait_limit",
+           "sattn_fwd_quantized_sparse", "sattn_fwd_sparse")
 
 
 class SattnError(RuntimeError):
@@ -78,6 +79,10 @@ def lib():
         L.sattn_kernel_launches.argtypes = [i]
         L.sattn_debug_set_wait_limit.restype = i
         L.sattn_debug_set_wait_limit.argtypes = [ctypes.c_longlong, i]
+        L.sattn_fwd_quantized_sparse.restype = i
+        L.sattn_fwd_quantized_sparse.argtypes = [vp, sz, vp, i, i, i, i, i, f, i, vp, vp]
+        L.sattn_fwd_sparse.restype = i
+        L.sattn_fwd_sparse.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp]
         _lib = L
     return _lib
 
@@ -162,6 +167,45 @@ def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None
                            int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype, q_per_token),
                            _stream(stream)),
            "sattn_fwd")
+    return out
+
+
+def _check_block_mask(block_mask, q):
+    B, H, N, _ = q.shape
+    nb = (N + 127) // 128
+    if not block_mask.is_cuda or block_mask.dtype not in (torch.uint8, torch.bool):
+        raise ValueError("block_mask must be a CUDA uint8/bool tensor")
+    if tuple(block_mask.shape) != (B, H, nb, nb) or not block_mask.is_contiguous():
+        raise ValueError(f"block_mask must be contiguous [B, H, {nb}, {nb}]")
+
+
+def fwd_sparse(q, k, v, block_mask, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None,
+               q_per_token=False):
+    """``fwd`` that skips the 128 x 128 (query, key) blocks where ``block_mask``
+    [B, H, ceil(N/128), ceil(N/128)] (uint8 or bool, on the device) is 0."""
+    B, H, N, d = _check_qkv(q, k, v)
+    _check_block_mask(block_mask, q)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().sattn_fwd_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
+                                  int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype, q_per_token),
+                                  block_mask.data_ptr(), _stream(stream)),
+           "sattn_fwd_sparse")
+    return out
+
+
+def fwd_quantized_sparse(workspace, shape, block_mask, causal=False, sm_scale=None, mode="i8f8",
+                         dtype=torch.bfloat16, out=None, stream=None, q_per_token=False):
+    """``fwd_quantized`` with block-sparse key skipping (see ``fwd_sparse``)."""
+    B, H, N, d = shape
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=dtype, device=workspace.device)
+    _check_block_mask(block_mask, out)
+    _check(lib().sattn_fwd_quantized_sparse(workspace.data_ptr(), workspace.numel(), out.data_ptr(),
+                                            B, H, N, d, int(bool(causal)), float(sm_scale or 0.0),
+                                            mode_code(mode, dtype, q_per_token), block_mask.data_ptr(),
+                                            _stream(stream)),
+           "sattn_fwd_quantized_sparse")
     return out
 
 

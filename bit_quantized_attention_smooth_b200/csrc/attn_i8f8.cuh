@@ -79,7 +79,12 @@ struct AttnArgs {
   int sq_stride;     // nblk, or N when q_per_token
   int q_per_token;   // 1: one Q scale per token
   float sm_log2;     // sm_scale * log2(e)
+  const uint8_t *block_mask;   // [BH, nblk, nblk], nonzero = keep the 128x128 block; nullptr = dense
 };
+
+// Largest key-tile count of a block-sparse call: the CTA keeps its query
+// tiles' rows of the block mask in shared memory.
+constexpr int kMaxMaskTiles = 2048;
 
 template <int D>
 struct AttnSmem {
@@ -91,7 +96,8 @@ struct AttnSmem {
   static constexpr int kK = kQ + kQTiles * kQBytes;              // [stages]
   static constexpr int kV = kK + kKVStages * kKBytes;            // [stages]
   static constexpr int kP = kV + kKVStages * kVBytes;            // [2 tiles][2 buffers]
-  static constexpr int kBar = kP + kQTiles * 2 * kPBytes;
+  static constexpr int kMask = kP + kQTiles * 2 * kPBytes;       // [2 tiles][kMaxMaskTiles] bytes (block-sparse calls)
+  static constexpr int kBar = kMask + kQTiles * kMaxMaskTiles;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
   // p_full[2][2], pv_done[2][2], drain
   static constexpr int kNumBars = 1 + 4 * kKVStages + 2 + 2 + 4 + 4 + 1;
@@ -205,7 +211,7 @@ __device__ __forceinline__ float p_pass(uint32_t s_tmem, float c, float b, uint8
   return tsum2.x + tsum2.y;
 }
 
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool SPARSE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
@@ -245,8 +251,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     nkv_of[x] = qt_of[x] >= nkv_all ? 0 : (CAUSAL ? min(qt_of[x] + 1, nkv_all) : nkv_all);
   }
   const int nkv_max = max(nkv_of[0], nkv_of[1]);
+  // Block-sparse skipping: key tile j of query tile x is processed iff
+  // need(x, j).  The three roles walk the same sequences: the producer and the
+  // MMA issuer the tiles that either query tile needs (the K/V ring advances
+  // per such tile), each softmax warpgroup the tiles its query tile needs (its
+  // S, P and O_in barriers advance per such tile).  Dense calls need every
+  // tile below nkv_of[x], and the sequences are the tile indices.
+  const uint8_t *smask = smem + L::kMask;
+  auto need = [&](int x, int j) -> bool { return j < nkv_of[x] && (!SPARSE || smask[x * kMaxMaskTiles + j] != 0); };
 
   // ------------------------------------------------------------ set-up
+  if (SPARSE) {
+    uint8_t *sm = smem + L::kMask;
+    for (int i = tid; i < kQTiles * nkv_all; i += kAttnThreads) {
+      const int x = i / nkv_all, j = i - x * nkv_all;
+      sm[x * kMaxMaskTiles + j] = qt_of[x] < nkv_all
+          ? args.block_mask[(static_cast<size_t>(bh) * nkv_all + qt_of[x]) * nkv_all + j] : uint8_t(0);
+    }
+  }
   if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -286,35 +308,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp == 8) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int last_j = -1;
+      int last_u = -1;
       const int withheld = g_withhold_k_tile;            // -1 except under the failure-path test hook
       const int nq = nkv_of[1] > 0 ? 2 : 1;             // tile B may lie past the last token
       mbar_arrive_expect_tx(q_full, nq * L::kQBytes);
       for (int x = 0; x < nq; ++x)
         tma_load_3d(smem + L::kQ + x * L::kQBytes, &tm_q, q_full, 0, qt_of[x] * kTile, bh);
-      for (int j = 0; j < nkv_max; ++j) {
-        const int s = j % kKVStages;
-        const uint32_t ph = (j / kKVStages) & 1;
+      for (int j = 0, un = 0; j < nkv_max; ++j) {       // un: position in the sequence of loaded tiles
+        if (SPARSE && !need(0, j) && !need(1, j)) continue;
+        const int u = SPARSE ? un : j;                     // dense: every tile below nkv_max is loaded
+        const int s = u % kKVStages;
+        const uint32_t ph = (u / kKVStages) & 1;
         if (!mbar_wait(&k_empty[s], ph ^ 1, abort_flag)) break;
-        if (j != withheld) {
+        if (u != withheld) {
           mbar_arrive_expect_tx(&k_full[s], L::kKBytes);
           tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
         }
         if (!mbar_wait(&v_empty[s], ph ^ 1, abort_flag)) {
-          if (j != withheld) drain_wait(&k_full[s], ph);   // K_j is in flight without its V_j
+          if (u != withheld) drain_wait(&k_full[s], ph);   // K_j is in flight without its V_j
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kVBytes);
         tma_load_3d(smem + L::kV + s * L::kVBytes, &tm_v, &v_full[s], j * kTile, 0, bh);
-        last_j = j;
+        last_u = u;
+        ++un;
       }
       if (*abort_flag) {
         // Wait for every copy this thread issued before the CTA releases its smem.
         drain_wait(q_full, 0);
-        for (int j = max(0, last_j - kKVStages + 1); j <= last_j; ++j) {
-          const uint32_t ph = (j / kKVStages) & 1;
-          if (j != withheld) drain_wait(&k_full[j % kKVStages], ph);
-          drain_wait(&v_full[j % kKVStages], ph);
+        for (int u = max(0, last_u - kKVStages + 1); u <= last_u; ++u) {
+          const uint32_t ph = (u / kKVStages) & 1;
+          if (u != withheld) drain_wait(&k_full[u % kKVStages], ph);
+          drain_wait(&v_full[u % kKVStages], ph);
         }
       }
     }
@@ -325,17 +350,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       constexpr uint32_t kIdescQK = idesc_i8_s32(kTile, kTile);
       constexpr uint32_t kIdescPV = idesc_e4m3_f32(kTile, D);
       bool ok = mbar_wait(q_full, 0, abort_flag);
+      int u = 0, prev_u = -1, prev_j = -1;               // loaded-tile sequence: this and the previous tile
+      int nqk[kQTiles] = {0, 0}, npv[kQTiles] = {0, 0};  // per query tile: QK and PV products issued
       for (int j = 0; ok && j <= nkv_max; ++j) {
+        const bool tail = j == nkv_max;                   // one step past the last tile: its P V only
+        if (SPARSE && !tail && !need(0, j) && !need(1, j)) continue;
+        if (!SPARSE) {                                     // dense: the sequences are the tile indices
+          u = j;
+          prev_u = prev_j = j - 1;
+          nqk[0] = nqk[1] = j;
+          npv[0] = npv[1] = j - 1;
+        }
         bool k_ready = false, v_ready = false;
 #pragma unroll
         for (int x = 0; x < kQTiles && ok; ++x) {
-          if (j < nkv_of[x]) {                              // S_x = Q_x K_j^T
-            const int s = j % kKVStages;
+          if (!tail && need(x, j)) {                        // S_x = Q_x K_j^T
+            const int s = u % kKVStages;
             if (!k_ready) {
-              ok = mbar_wait(&k_full[s], (j / kKVStages) & 1, abort_flag);
+              ok = mbar_wait(&k_full[s], (u / kKVStages) & 1, abort_flag);
               k_ready = true;
             }
-            ok = ok && mbar_wait(&s_free[x], (j & 1) ^ 1, abort_flag);
+            ok = ok && mbar_wait(&s_free[x], (nqk[x] & 1) ^ 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
             const uint32_t sQ = smem_u32(smem + L::kQ + x * L::kQBytes);
@@ -345,13 +380,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               mma_i8(tmem + x * kTile, sdesc_kmajor<D>(sQ + kk * 32), sdesc_kmajor<D>(sK + kk * 32), kIdescQK,
                      kk > 0 ? 1u : 0u);
             mma_commit(&s_full[x]);
+            ++nqk[x];
           }
-          if (j >= 1 && j - 1 < nkv_of[x]) {                // O_in_x (+)= P_x(j-1) V_{j-1}
-            const int t = j - 1;
-            const int s = t % kKVStages;
+          if (prev_u >= 0 && need(x, prev_j)) {             // O_in_x (+)= P_x V of the previous loaded tile
+            if (!SPARSE) npv[x] = prev_j;
+            const int t = npv[x];
+            const int s = prev_u % kKVStages;
             const int pb = x * 2 + (t & 1);
             if (!v_ready) {
-              ok = mbar_wait(&v_full[s], (t / kKVStages) & 1, abort_flag);
+              ok = mbar_wait(&v_full[s], (prev_u / kKVStages) & 1, abort_flag);
               v_ready = true;
             }
             ok = ok && mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag);
@@ -365,11 +402,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               mma_f8f6f4(tmem + kOin0 + x * D, sdesc_kmajor<128>(sP + kk * 32), sdesc_kmajor<128>(sV + kk * 32),
                          kIdescPV, acc | (kk > 0 ? 1u : 0u));
             mma_commit(&pv_done[pb]);
+            ++npv[x];
           }
         }
         if (!ok) break;
-        if (k_ready) mma_commit(&k_empty[j % kKVStages]);
-        if (v_ready) mma_commit(&v_empty[(j - 1) % kKVStages]);
+        if (k_ready) mma_commit(&k_empty[u % kKVStages]);
+        if (v_ready) mma_commit(&v_empty[prev_u % kKVStages]);
+        if (SPARSE && !tail) {
+          prev_u = u++;
+          prev_j = j;
+        }
       }
       if (!ok) {
         // Let every MMA issued so far finish before TMEM is released.
@@ -404,30 +446,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float beta = 1.f;          // the outer accumulator is beta * o_out (rescaled lazily)
     bool ok = true;
 
+    int n = 0;                 // key tiles processed (the S, P and O_in barriers advance per tile)
     for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(&s_full[x], j & 1, abort_flag)) { ok = false; break; }
+      if (SPARSE && !smask[x * kMaxMaskTiles + j]) continue;
+      if (!SPARSE) n = j;                                  // dense: the tile index
+      if (!mbar_wait(&s_full[x], n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const bool masked = ((j == nkv_all - 1) && (N & (kTile - 1))) || (CAUSAL && j == qt);
       const int kv0 = j * kTile;
       const float c = cq * sk[j];
 
-      // P~ -> E4M3 into P buffer (j & 1), once P V of tile j-2 has read it
-      const int pb = x * 2 + (j & 1);
-      if (!mbar_wait(&pv_done[pb], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      uint8_t *prow = p_base + (j & 1) * L::kPBytes;
+      // P~ -> E4M3 into P buffer (n & 1), once P V of the tile two before has read it
+      const int pb = x * 2 + (n & 1);
+      if (!mbar_wait(&pv_done[pb], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      uint8_t *prow = p_base + (n & 1) * L::kPBytes;
       // speculative pass with the current reference max (0 at the first tile,
       // which only serves to find the tile's row max)
-      const float m_try = j > 0 ? m_ref : 0.f;
+      const float m_try = n > 0 ? m_ref : 0.f;
       float2 xm2 = make_float2(-INFINITY, -INFINITY);
       float tsum = p_pass(s_tmem, c, m_try - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
       // x = S2 - m + log2 c_P;  the row max moves when S2max - m > tau  <=>  xmax > log2 448
       const float xmax = fmaxf(xm2.x, xm2.y);
-      const bool up = j == 0 || xmax > kLog2_448;
+      const bool up = n == 0 || xmax > kLog2_448;
       const bool moved = __any_sync(0xffffffffu, up);   // warp-uniform
       float m_new = m_ref, alpha = 1.f;
       if (moved) {
         if (up) m_new = fmaxf(m_ref, xmax + (m_try - kLog2_CP));   // the tile's row max
-        alpha = j > 0 ? ex2_approx(m_ref - m_new) : 0.f;
+        alpha = n > 0 ? ex2_approx(m_ref - m_new) : 0.f;
         tsum = p_pass(s_tmem, c, m_new - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
       }
       tc_fence_before();
@@ -436,10 +481,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       lsum = fmaf(alpha, lsum, tsum);
 
       // two-level accumulation: flush O_in at a group start, or rescale when the reference max moved
-      const bool boundary = j > 0 && (j % kFlushEvery) == 0;
-      const bool grow = j > 0 && moved;
+      const bool boundary = n > 0 && (n % kFlushEvery) == 0;
+      const bool grow = n > 0 && moved;
       if (boundary || grow) {
-        const int t = j - 1;
+        const int t = n - 1;
         if (!mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (boundary) {
@@ -490,11 +535,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[pb]);
       m_ref = m_new;
+      ++n;
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && nkv > 0) {
-      const int t = nkv - 1;
+    if (ok && n > 0) {
+      const int t = n - 1;
       if (mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) {
         tc_fence_after();
         const float inv_l = 1.f / lsum;
@@ -520,6 +566,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
       }
+    } else if (ok && qt < nkv_all && row_g < N) {
+      // every key block of this query tile is skipped: the rows are zeros
+      uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D);
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 

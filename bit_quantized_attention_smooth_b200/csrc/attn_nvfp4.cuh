@@ -53,6 +53,7 @@ struct AttnF4Args {
   int N;
   int nblk;
   float sm_log2;
+  const uint8_t *block_mask;   // [BH, nblk, nblk], nonzero = keep the 128x128 block; nullptr = dense
 };
 
 template <int D>
@@ -74,7 +75,8 @@ struct AttnF4Smem {
   static constexpr int kSfVo = kSfK + kKVStages * kSfQK;
   static constexpr int kSfPo = kSfVo + kKVStages * kSfV;
   static constexpr int kX = kSfPo + 2 * kSfP;          // float [2 phases][4 quarters][128] + [4][128]
-  static constexpr int kBar = kX + (2 * 4 * 128 + 4 * 128) * 4;
+  static constexpr int kMask = kX + (2 * 4 * 128 + 4 * 128) * 4;   // [kMaxMaskTiles] bytes (block-sparse calls)
+  static constexpr int kBar = kMask + kMaxMaskTiles;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
   // p_full[2], pv_done[2], quad[4], drain
   static constexpr int kNumBars = 1 + 4 * kKVStages + 8 + 4 + 1;
@@ -134,7 +136,7 @@ __device__ __forceinline__ uint64_t sdesc_f4(uint32_t smem_addr) {
          (uint64_t(1) << 46) | (mode << 61);
 }
 
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool SPARSE>
 __global__ void __launch_bounds__(kF4Threads, 1)
     attn_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const AttnF4Args args) {
@@ -177,6 +179,16 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   const int qt = CAUSAL ? (static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x))
                         : static_cast<int>(blockIdx.x);
   const int nkv = CAUSAL ? min(qt + 1, nkv_all) : nkv_all;
+  // Block-sparse skipping: key tile j is processed iff need(j); every role
+  // walks the same sequence of needed tiles, and the barriers and buffers
+  // advance per position n in it (n == j for dense calls).
+  const uint8_t *smask = smem + L::kMask;
+  auto need = [&](int jj) -> bool { return !SPARSE || smask[jj] != 0; };
+  if (SPARSE) {
+    uint8_t *sm = smem + L::kMask;
+    for (int i = tid; i < nkv_all; i += kF4Threads)
+      sm[i] = args.block_mask[(static_cast<size_t>(bh) * nkv_all + qt) * nkv_all + i];
+  }
 
   if (warp == 17) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -214,38 +226,39 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   if (warp == 16) {
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int last_j = -1;
+      int last_n = -1;
       const int withheld = g_withhold_k_tile;            // -1 except under the failure-path test hook
       const size_t sf_qk_tile = static_cast<size_t>(L::kSfQK);
       mbar_arrive_expect_tx(q_full, L::kQBytes + L::kSfQK);
       tma_load_3d(smem + L::kQ, &tm_q, q_full, 0, qt * kTile, bh);
       bulk_load(smem + L::kSfQ, args.sfq + (static_cast<size_t>(bh) * nkv_all + qt) * sf_qk_tile, L::kSfQK, q_full);
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % kKVStages;
-        const uint32_t ph = (j / kKVStages) & 1;
+      for (int j = 0, n = 0; j < nkv; ++j) {
+        if (!need(j)) continue;
+        const int s = n % kKVStages;
+        const uint32_t ph = (n / kKVStages) & 1;
         if (!mbar_wait(&k_empty[s], ph ^ 1, abort_flag)) break;
-        if (j != withheld) {
+        if (n != withheld) {
           mbar_arrive_expect_tx(&k_full[s], L::kKBytes + L::kSfQK);
           tma_load_3d(smem + L::kK + s * L::kKBytes, &tm_k, &k_full[s], 0, j * kTile, bh);
           bulk_load(smem + L::kSfK + s * L::kSfQK, args.sfk + (static_cast<size_t>(bh) * nkv_all + j) * sf_qk_tile,
                     L::kSfQK, &k_full[s]);
         }
         if (!mbar_wait(&v_empty[s], ph ^ 1, abort_flag)) {
-          if (j != withheld) drain_wait(&k_full[s], ph);
+          if (n != withheld) drain_wait(&k_full[s], ph);
           break;
         }
         mbar_arrive_expect_tx(&v_full[s], L::kVBytes + L::kSfV);
         tma_load_3d(smem + L::kV + s * L::kVBytes, &tm_v, &v_full[s], j * (kTile / 2), 0, bh);
         bulk_load(smem + L::kSfVo + s * L::kSfV, args.sfv + (static_cast<size_t>(bh) * nkv_all + j) * L::kSfV,
                   L::kSfV, &v_full[s]);
-        last_j = j;
+        last_n = n++;
       }
       if (*abort_flag) {
         drain_wait(q_full, 0);
-        for (int j = max(0, last_j - kKVStages + 1); j <= last_j; ++j) {
-          const uint32_t ph = (j / kKVStages) & 1;
-          if (j != withheld) drain_wait(&k_full[j % kKVStages], ph);
-          drain_wait(&v_full[j % kKVStages], ph);
+        for (int n = max(0, last_n - kKVStages + 1); n <= last_n; ++n) {
+          const uint32_t ph = (n / kKVStages) & 1;
+          if (n != withheld) drain_wait(&k_full[n % kKVStages], ph);
+          drain_wait(&v_full[n % kKVStages], ph);
         }
       }
     }
@@ -263,12 +276,13 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         for (int kk = 0; kk < kNK; ++kk)
           tmem_cp_sf(tmem + kSfQc + 4 * kk, sdesc_sf_block(smem_u32(smem + L::kSfQ + 512 * kk)));
       }
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int s = j % kKVStages;
-          const int b = j & 1;
-          ok = mbar_wait(&k_full[s], (j / kKVStages) & 1, abort_flag) &&
-               mbar_wait(&s_free[b], ((j >> 1) & 1) ^ 1, abort_flag);
+      for (int j = 0, n = 0; ok && j <= nkv; ++j) {
+        if (j < nkv && !need(j)) continue;
+        if (j < nkv) {                                    // S_b = Q K_j^T, the n-th needed tile
+          const int s = n % kKVStages;
+          const int b = n & 1;
+          ok = mbar_wait(&k_full[s], (n / kKVStages) & 1, abort_flag) &&
+               mbar_wait(&s_free[b], ((n >> 1) & 1) ^ 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sK = smem_u32(smem + L::kK + s * L::kKBytes);
@@ -283,8 +297,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           mma_commit(&s_full[b]);
           mma_commit(&k_empty[s]);
         }
-        if (j > 0) {
-          const int t = j - 1;
+        if (n > 0) {                                      // O_in = P V of the (n-1)-th needed tile
+          const int t = n - 1;
           const int s = t % kKVStages;
           const int b = t & 1;
           ok = mbar_wait(&v_full[s], (t / kKVStages) & 1, abort_flag) &&
@@ -307,6 +321,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           mma_commit(&pv_done[b]);
           mma_commit(&v_empty[s]);
         }
+        ++n;
       }
       if (!ok) {
         mma_commit(drain_bar);
@@ -341,9 +356,11 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       }
     };
 
+    int n = 0;                                        // key tiles processed
     for (int j = 0; j < nkv && ok; ++j) {
-      const int b = j & 1;
-      if (!mbar_wait(&s_full[b], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!need(j)) continue;
+      const int b = n & 1;
+      if (!mbar_wait(&s_full[b], (n >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       uint32_t sa[32];
       tmem_ld_32x32b_x32(tmem + lane_base + b * kTile + kq * 32, sa);
@@ -370,11 +387,11 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         t[5] = __uint_as_float(v[15]);
         bmax[hb] = fmaxf(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]));
       }
-      float *xm = xmax + (j & 1) * 4 * 128;
+      float *xm = xmax + (n & 1) * 4 * 128;
       xm[kq * 128 + r] = fmaxf(bmax[0], bmax[1]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&quad[wq]);
-      if (!mbar_wait(&quad[wq], j & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&quad[wq], n & 1, abort_flag)) { ok = false; break; }
       const float tmax = fmaxf(fmax3(xm[r], xm[128 + r], xm[256 + r]), xm[384 + r]);
       const float m_tile = tmax * cl;                   // finite: every processed tile has a valid key
       const float m_new = fmaxf(m_ref, m_tile);
@@ -384,7 +401,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       const float moff6 = moff + kLog2_6;
 
       // two-stage NVFP4 quantisation of this quarter of P into buffer b
-      if (!mbar_wait(&pv_done[b], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&pv_done[b], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       uint8_t *prow = smem + L::kP + b * L::kPBytes + r * 64;
       uint8_t *psf = smem + L::kSfPo + b * L::kSfP + (kq >> 1) * 512;   // 64-key slice of the quarter
       float psum = 0.f;
@@ -428,8 +445,8 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       *reinterpret_cast<uint4 *>(prow + ((kq ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
 
       // flush the previous tile: O_out = a O_out + s1 O_in (this quarter of the columns)
-      if (j > 0) {
-        const int t = j - 1;
+      if (n > 0) {
+        const int t = n - 1;
         if (!mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint32_t o[kQD];
@@ -451,15 +468,16 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
       m_ref = m_new;
+      ++n;
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && nkv > 0) {
+    if (ok && n > 0) {
       xl[kq * 128 + r] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&quad[wq]);
-      const int t = nkv - 1;
-      if (mbar_wait(&quad[wq], nkv & 1, abort_flag) && mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) {
+      const int t = n - 1;
+      if (mbar_wait(&quad[wq], n & 1, abort_flag) && mbar_wait(&pv_done[t & 1], (t >> 1) & 1, abort_flag)) {
         tc_fence_after();
         const float inv_l = 1.f / ((xl[r] + xl[128 + r]) + (xl[256 + r] + xl[384 + r]));
         OutT *orow = reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D + kq * kQD;
@@ -479,6 +497,12 @@ __global__ void __launch_bounds__(kF4Threads, 1)
             dst[u] = make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
         }
       }
+    } else if (ok && row_g < N) {
+      // every key block of this query tile is skipped: the rows are zeros
+      uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<OutT *>(args.out) + (static_cast<size_t>(bh) * N + row_g) * D +
+                                             kq * kQD);
+#pragma unroll
+      for (int u = 0; u < kQD / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 

@@ -181,9 +181,9 @@ int launch_quant_nvfp4(const void *q, const void *k, const void *v, int BH, int 
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool SPARSE>
 int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
-                      cudaStream_t st) {
+                      const uint8_t *block_mask, cudaStream_t st) {
   using SL = AttnF4Smem<D>;
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle swqk = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
@@ -196,7 +196,7 @@ int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, 
   // More than half of the SM's shared memory: one CTA (and its 512 TMEM
   // columns) per SM.
   const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
-  auto kern = attn_nvfp4_kernel<D, CAUSAL, OutT>;
+  auto kern = attn_nvfp4_kernel<D, CAUSAL, OutT, SPARSE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SATTN_ERR_CUDA;
   AttnF4Args a;
@@ -207,14 +207,15 @@ int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, 
   a.N = N;
   a.nblk = L.nblk;
   a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  a.block_mask = block_mask;
   kern<<<dim3(L.nblk, BH), kF4Threads, smem, st>>>(tq, tk, tv, a);
   g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL, typename OutT>
+template <int D, bool CAUSAL, typename OutT, bool SPARSE>
 int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
-                     bool per_token, cudaStream_t st) {
+                     bool per_token, const uint8_t *block_mask, cudaStream_t st) {
   using SL = AttnSmem<D>;
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle swqk = D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -226,7 +227,7 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
   // More than half of the SM's shared memory: one CTA (and its 512 TMEM
   // columns) per SM.
   const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
-  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT>;
+  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, SPARSE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SATTN_ERR_CUDA;
   // The kernel's setmaxnreg split must fit in its launch registers, or its
@@ -244,6 +245,7 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
   a.sq_stride = per_token ? N : L.nblk;
   a.q_per_token = per_token ? 1 : 0;
   a.sm_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  a.block_mask = block_mask;
   kern<<<dim3((L.nblk + kQTiles - 1) / kQTiles, BH), kAttnThreads, smem, st>>>(tq, tk, tv, a);
   g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
@@ -251,13 +253,50 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
 
 template <int D, typename OutT>
 int dispatch_attn(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, int causal, float sm,
-                  int mode, cudaStream_t st) {
-  if (is_nvfp4(mode))
-    return causal ? launch_attn_nvfp4<D, true, OutT>(ws, L, out, BH, N, sm, st)
-                  : launch_attn_nvfp4<D, false, OutT>(ws, L, out, BH, N, sm, st);
+                  int mode, const uint8_t *mask, cudaStream_t st) {
+  if (is_nvfp4(mode)) {
+    if (mask != nullptr)
+      return causal ? launch_attn_nvfp4<D, true, OutT, true>(ws, L, out, BH, N, sm, mask, st)
+                    : launch_attn_nvfp4<D, false, OutT, true>(ws, L, out, BH, N, sm, mask, st);
+    return causal ? launch_attn_nvfp4<D, true, OutT, false>(ws, L, out, BH, N, sm, nullptr, st)
+                  : launch_attn_nvfp4<D, false, OutT, false>(ws, L, out, BH, N, sm, nullptr, st);
+  }
   const bool pt = q_per_token(mode);
-  return causal ? launch_attn_i8f8<D, true, OutT>(ws, L, out, BH, N, sm, pt, st)
-                : launch_attn_i8f8<D, false, OutT>(ws, L, out, BH, N, sm, pt, st);
+  if (mask != nullptr)
+    return causal ? launch_attn_i8f8<D, true, OutT, true>(ws, L, out, BH, N, sm, pt, mask, st)
+                  : launch_attn_i8f8<D, false, OutT, true>(ws, L, out, BH, N, sm, pt, mask, st);
+  return causal ? launch_attn_i8f8<D, true, OutT, false>(ws, L, out, BH, N, sm, pt, nullptr, st)
+                : launch_attn_i8f8<D, false, OutT, false>(ws, L, out, BH, N, sm, pt, nullptr, st);
+}
+
+// Checks of a block-sparse call beyond those of the dense one.
+int check_block_mask(int N, const void *block_mask) {
+  if (block_mask == nullptr) return SATTN_ERR_INVALID_ARG;
+  if ((N + kTile - 1) / kTile > kMaxMaskTiles) return SATTN_ERR_UNSUPPORTED;
+  return SATTN_OK;
+}
+
+int fwd_quantized_impl(const void *workspace, size_t ws_bytes, void *out, int B, int H, int N, int d, int causal,
+                       float sm_scale, int mode, const uint8_t *mask, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (!aligned16(out)) return SATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
+  const sattn_ws_layout_t L = make_layout(B, H, N, d, mode);
+  if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
+  const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+  if (static_cast<const uint8_t *>(out) < ws + L.total &&
+      ws < static_cast<const uint8_t *>(out) + static_cast<size_t>(B) * H * N * d * 2)
+    return SATTN_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) sm_scale = 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const bool fp16 = (mode & SATTN_FP16_IO) != 0;
+  if (d == 128)
+    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, mode, mask, cs)
+                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, mode, mask, cs);
+  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, mode, mask, cs)
+              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, mode, mask, cs);
 }
 
 // Library-owned workspace of sattn_fwd, one per device.
@@ -317,29 +356,21 @@ int sattn_quantize(const void *q, const void *k, const void *v, int B, int H, in
 
 int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B, int H, int N, int d, int causal,
                         float sm_scale, int mode, sattn_stream_t stream) {
-  const int st = check_shape(B, H, N, d, mode);
-  if (st != SATTN_OK) return st;
-  if (!aligned16(out)) return SATTN_ERR_INVALID_ARG;
-  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
-  const sattn_ws_layout_t L = make_layout(B, H, N, d, mode);
-  if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
-  const uint8_t *ws = static_cast<const uint8_t *>(workspace);
-  if (static_cast<const uint8_t *>(out) < ws + L.total &&
-      ws < static_cast<const uint8_t *>(out) + static_cast<size_t>(B) * H * N * d * 2)
-    return SATTN_ERR_INVALID_ARG;
-  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) sm_scale = 1.0f / std::sqrt(static_cast<float>(d));
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const int BH = B * H;
-  const bool fp16 = (mode & SATTN_FP16_IO) != 0;
-  if (d == 128)
-    return fp16 ? dispatch_attn<128, __half>(ws, L, out, BH, N, causal, sm_scale, mode, cs)
-                : dispatch_attn<128, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, mode, cs);
-  return fp16 ? dispatch_attn<64, __half>(ws, L, out, BH, N, causal, sm_scale, mode, cs)
-              : dispatch_attn<64, __nv_bfloat16>(ws, L, out, BH, N, causal, sm_scale, mode, cs);
+  return fwd_quantized_impl(workspace, ws_bytes, out, B, H, N, d, causal, sm_scale, mode, nullptr, stream);
 }
 
-int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
-              float sm_scale, int mode, sattn_stream_t stream) {
+int sattn_fwd_quantized_sparse(const void *workspace, size_t ws_bytes, void *out, int B, int H, int N, int d,
+                               int causal, float sm_scale, int mode, const uint8_t *block_mask,
+                               sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  const int sm = check_block_mask(N, block_mask);
+  if (sm != SATTN_OK) return sm;
+  return fwd_quantized_impl(workspace, ws_bytes, out, B, H, N, d, causal, sm_scale, mode, block_mask, stream);
+}
+
+static int fwd_impl(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
+                    float sm_scale, int mode, const uint8_t *mask, sattn_stream_t stream) {
   const int st = check_shape(B, H, N, d, mode);
   if (st != SATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SATTN_ERR_INVALID_ARG;
@@ -370,7 +401,21 @@ int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int
   }
   const int s1 = sattn_quantize(q, k, v, B, H, N, d, mode, ws, ws_bytes, stream);
   if (s1 != SATTN_OK) return s1;
-  return sattn_fwd_quantized(ws, ws_bytes, out, B, H, N, d, causal, sm_scale, mode, stream);
+  return fwd_quantized_impl(ws, ws_bytes, out, B, H, N, d, causal, sm_scale, mode, mask, stream);
+}
+
+int sattn_fwd(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
+              float sm_scale, int mode, sattn_stream_t stream) {
+  return fwd_impl(q, k, v, out, B, H, N, d, causal, sm_scale, mode, nullptr, stream);
+}
+
+int sattn_fwd_sparse(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int causal,
+                     float sm_scale, int mode, const uint8_t *block_mask, sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  const int sm = check_block_mask(N, block_mask);
+  if (sm != SATTN_OK) return sm;
+  return fwd_impl(q, k, v, out, B, H, N, d, causal, sm_scale, mode, block_mask, stream);
 }
 
 // Pipelined forward over host buffers: chunks of heads are copied in on one

@@ -118,6 +118,22 @@ int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out,
                         int B, int H, int N, int d, int causal, float sm_scale,
                         int mode, sattn_stream_t stream);
 
+/* Block-sparse sattn_fwd_quantized: the 128 x 128 blocks of (query, key)
+ * that `block_mask` marks 0 are skipped -- their keys are left out of the
+ * softmax of that block's queries, and their K/V tiles are neither loaded nor
+ * multiplied -- on top of the causal mask (the "skip" part of Sparse-Linear
+ * Attention, TurboDiffusion explainer, SLA section, with the mask given by
+ * the caller).  block_mask: device memory, uint8 [B*H][nblk][nblk], nblk =
+ * ceil(N / 128), entry [bh][i][j] nonzero = query block i keeps key block j.
+ * A query block that keeps no key block gets zero output rows.  Both modes;
+ * nblk <= 2048 (N <= 262144), else SATTN_ERR_UNSUPPORTED; block_mask == NULL
+ * is SATTN_ERR_INVALID_ARG.  The
+ * mask is read by the kernel, so it must stay unchanged until `stream` has
+ * passed the call.  Otherwise as sattn_fwd_quantized. */
+int sattn_fwd_quantized_sparse(const void *workspace, size_t ws_bytes, void *out,
+                               int B, int H, int N, int d, int causal, float sm_scale,
+                               int mode, const uint8_t *block_mask, sattn_stream_t stream);
+
 /* sattn_quantize followed by sattn_fwd_quantized, with a workspace that the
  * library owns: the one-call, drop-in form of the attention (tag page,
  * SageAttention3 summary, bullet [5]: plug-and-play; explainer, section 1:
@@ -129,6 +145,13 @@ int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out,
 int sattn_fwd(const void *q, const void *k, const void *v, void *out,
               int B, int H, int N, int d, int causal, float sm_scale, int mode,
               sattn_stream_t stream);
+
+/* sattn_fwd with block-sparse key skipping (block_mask as in
+ * sattn_fwd_quantized_sparse).  The quantization is the dense one: the K
+ * mean and the V channel scales still cover every token. */
+int sattn_fwd_sparse(const void *q, const void *k, const void *v, void *out,
+                     int B, int H, int N, int d, int causal, float sm_scale, int mode,
+                     const uint8_t *block_mask, sattn_stream_t stream);
 
 /* sattn_fwd on HOST buffers (a deployment variant; the pages have no
  * counterpart): q, k, v and out are host pointers ([B, H, N, d],

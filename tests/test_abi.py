@@ -135,3 +135,16 @@ def test_per_token_q_layout(L):
     assert tok["total"] == L.sattn_workspace_bytes(2, 3, 1000, 128, QTOK)
     assert L.sattn_workspace_bytes(2, 3, 1000, 128, NVFP4 | QTOK) == 0
     assert L.sattn_workspace_bytes(2, 3, 1000, 128, 0x400) == 0
+
+
+def test_block_sparse_entry_points_validate_before_any_cuda_call(L):
+    p = ctypes.c_void_p(1 << 20)
+    o = ctypes.c_void_p(1 << 40)
+    m = ctypes.c_void_p(1 << 30)
+    f = L.sattn_fwd_sparse
+    assert f(p, p, p, o, 1, 2, 1000, 128, 0, 0.0, BF16, None, None) == INVALID       # no mask
+    assert f(p, p, p, o, 1, 1, 262145, 64, 0, 0.0, BF16, m, None) == UNSUPPORTED     # more than 2048 key tiles
+    assert f(p, p, p, o, 1, 2, 1000, 96, 0, 0.0, BF16, m, None) == UNSUPPORTED       # head dim
+    g = L.sattn_fwd_quantized_sparse
+    assert g(p, 1 << 30, o, 1, 2, 1000, 128, 0, 0.0, BF16, None, None) == INVALID
+    assert g(None, 1 << 30, o, 1, 2, 1000, 128, 0, 0.0, BF16, m, None) == WORKSPACE
