@@ -143,11 +143,15 @@ def oracle_sample(w, target_s, rows_n=None):
         return 4.0 * rows_n * w.N * w.d, time.perf_counter() - t0, rows_n
     emul(qf, kf, vf, rows=np.arange(1))            # warm caches
     t0 = time.perf_counter()
-    emul(qf, kf, vf, rows=np.arange(65))
-    t65 = time.perf_counter() - t0
-    # linear through the origin: over-estimates the per-row cost (the time
-    # includes the head's quantisation), so the sample stays within target_s
-    rows_n = int(max(1, min(w.N, 65 * target_s / t65)))
+    emul(qf, kf, vf, rows=np.arange(64))
+    t64 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    emul(qf, kf, vf, rows=np.arange(320))
+    t320 = time.perf_counter() - t0
+    # fixed cost (the head's quantisation) plus a cost per row, fitted on two sizes
+    per_row = max((t320 - t64) / 256, 1e-6)
+    fixed = max(t64 - 64 * per_row, 0.0)
+    rows_n = int(max(1, min(w.N, (target_s - fixed) / per_row)))
     rows = np.linspace(0, w.N - 1, rows_n).astype(np.int64)
     t0 = time.perf_counter()
     emul(qf, kf, vf, rows=rows)
