@@ -119,6 +119,27 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+// The current CUDA context (driver handle), looked up like the encoder above.
+// The library's per-device caches (owned workspace, host pipeline, address of
+// the no-alloc array) remember the context they were made in: after
+// cudaDeviceReset, or under another context, they are rebuilt instead of
+// reused (the old pointers died with their context and are not freed).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 // 3-D uint8 tensor [dim2][dim1][dim0] (dim0 contiguous), box {box0, box1, 1}.
 bool make_map_u8(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint64_t stride1,
                  uint64_t stride2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
@@ -303,6 +324,7 @@ int fwd_quantized_impl(const void *workspace, size_t ws_bytes, void *out, int B,
 struct OwnedWorkspace {
   void *ptr = nullptr;
   size_t bytes = 0;
+  CUcontext ctx = nullptr;   // context the pointer belongs to
 };
 std::mutex g_ws_mutex;
 OwnedWorkspace g_ws[kMaxDevices];
@@ -389,6 +411,8 @@ static int fwd_impl(const void *q, const void *k, const void *v, void *out, int 
   {
     std::lock_guard<std::mutex> lock(g_ws_mutex);
     OwnedWorkspace &w = g_ws[dev];
+    const CUcontext ctx = current_context();
+    if (w.ctx != ctx) w = OwnedWorkspace{nullptr, 0, ctx};   // a reset or another context: start afresh
     if (w.bytes < need) {
       if (w.ptr != nullptr && cudaFreeAsync(w.ptr, cs) != cudaSuccess) return SATTN_ERR_CUDA;
       w.ptr = nullptr;
@@ -427,6 +451,7 @@ int sattn_fwd_sparse(const void *q, const void *k, const void *v, void *out, int
 namespace {
 struct HostPipe {
   bool ready = false;
+  CUcontext ctx = nullptr;   // context the streams, events and buffers belong to
   cudaStream_t s_in = nullptr, s_out = nullptr, s_comp[2] = {nullptr, nullptr};
   cudaEvent_t ev_start = nullptr, ev_in[2] = {nullptr, nullptr}, ev_comp[2] = {nullptr, nullptr},
               ev_out[2] = {nullptr, nullptr};
@@ -510,6 +535,11 @@ int sattn_fwd_host(const void *q, const void *k, const void *v, void *out, int B
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(g_host_mutex);
   HostPipe &p = g_host[dev];
+  const CUcontext ctx = current_context();
+  if (p.ctx != ctx) {                     // a reset or another context: the old handles are gone
+    p = HostPipe{};
+    p.ctx = ctx;
+  }
   if (!host_pipe_init(p) || !host_pipe_reserve(p, 4 * part, ws_need)) return SATTN_ERR_CUDA;
   // everything this call does follows the caller's earlier work on its stream
   if (cudaEventRecord(p.ev_start, cs) != cudaSuccess) return SATTN_ERR_CUDA;
@@ -608,6 +638,7 @@ __device__ __align__(256) uint8_t g_noalloc_workspace[SATTN_NOALLOC_MAX_BYTES];
 namespace {
 std::mutex g_noalloc_mutex;
 void *g_noalloc_addr[kMaxDevices];   // device address of the array per device, once looked up
+CUcontext g_noalloc_ctx[kMaxDevices];  // context it was looked up in
 }  // namespace
 }  // namespace sattn
 
@@ -629,11 +660,13 @@ extern "C" int sattn_fwd_noalloc(const void *q, const void *k, const void *v, vo
   void *ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_addr[dev] == nullptr) {
+    const CUcontext ctx = current_context();
+    if (g_noalloc_addr[dev] == nullptr || g_noalloc_ctx[dev] != ctx) {
       void *addr = nullptr;
       if (cudaGetSymbolAddress(&addr, g_noalloc_workspace) != cudaSuccess || addr == nullptr)
         return SATTN_ERR_CUDA;
       g_noalloc_addr[dev] = addr;
+      g_noalloc_ctx[dev] = ctx;
     }
     ws = g_noalloc_addr[dev];
   }

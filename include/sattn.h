@@ -140,7 +140,9 @@ int sattn_fwd_quantized_sparse(const void *workspace, size_t ws_bytes, void *out
  * usable in place of FlashAttention).  One workspace per device, allocated on
  * first use with cudaMallocAsync on `stream` and grown (never shrunk) when a
  * larger problem arrives.  Calls that share a device must be ordered (same
- * stream, or synchronized), because they share this workspace.  `out` must
+ * stream, or synchronized), because they share this workspace, which belongs
+ * to the context current at its allocation (after cudaDeviceReset, or under
+ * another context, the next call allocates a new one).  `out` must
  * not alias q, k or v (SATTN_ERR_INVALID_ARG). */
 int sattn_fwd(const void *q, const void *k, const void *v, void *out,
               int B, int H, int N, int d, int causal, float sm_scale, int mode,
@@ -192,7 +194,9 @@ int sattn_fwd_host(const void *q, const void *k, const void *v, void *out,
  * SATTN_ERR_WORKSPACE, before any launch, when the problem needs more than
  * SATTN_NOALLOC_MAX_BYTES (sattn_workspace_bytes tells).  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture.  All calls
+ * device current, and so does the first call after the device's context
+ * changed (cudaDeviceReset, or the caller's own context); make such a call
+ * before any stream capture.  All calls
  * on one device share the array, which keeps the previous call's contents
  * (each call re-clears what must start at zero): calls that overlap on the GPU,
  * from other streams or host threads, race and must be ordered by the caller. */
