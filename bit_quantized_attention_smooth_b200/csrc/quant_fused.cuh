@@ -1,0 +1,340 @@
+// The quantiser: one persistent kernel for every tile of Q, K and V of both
+// modes.
+//
+// K smoothing needs the column mean of all of K before any K code, and the
+// per-channel V scale the column maximum of all of V before any V code, so K
+// and V are read twice: once for the statistics, once for the codes.  The
+// work is one queue of items, taken in ticket order by all CTAs; per head h:
+//   A(h) = statistics items of K (and, I8QK_F8PV, V) of h, then Q tiles of h
+//   B(h) = K tiles of h, then V tiles of h
+// A tile is 128 tokens x d of one tensor of one (b,h); a statistics item is
+// kStatBlocks consecutive tiles, reduced over the CTA and published once.
+// The order is A(0) A(1) B(0) A(2) B(1) ... A(BH-1) B(BH-2) B(BH-1): a head's
+// K and V are quantised about one head after their statistics were read, so
+// that their second read comes from L2 (two heads' K and V, about 34 MB at
+// N = 32760, d = 128, stay resident in the 126 MB L2; the statistics reads
+// carry an evict-last hint and every other read evict-first).  HBM then sees
+// each input byte once.
+//
+// A K or V tile waits for its head's statistics: at the end of every
+// statistics item, each of the d/32 warps that add into the head's
+// accumulators fences its atomics and bumps done[h] once; before the K/V tile
+// is handed to the compute warps, the producer spins (bounded) until done[h]
+// reaches d/32 times the head's number of statistics items.  The queue order
+// makes the wait finite: an item waits only for items with smaller tickets,
+// each already taken by a running CTA that processes its items in ticket
+// order (the tiles of one item in consecutive stages); the unfinished item
+// with the smallest ticket never waits.
+//
+// CTA: 8 compute warps + 1 producer warp.  The producer warp takes tickets,
+// bulk-copies (cp.async.bulk, no multicast) each tile into a ring of
+// kQuantStages shared-memory stages and, for a K or V tile, waits for the
+// head's statistics and puts the per-channel mu or s_v beside the stage; the
+// compute warps process the stages in order and release each with one arrive
+// per warp.  Two CTAs per SM.
+#pragma once
+
+#include "quant_i8f8.cuh"
+#include "quant_nvfp4.cuh"
+
+namespace sattn {
+
+constexpr int kQuantStages = 3;
+constexpr int kQuantThreads = kQuantConsumers + 32;
+constexpr int kStatBlocks = 4;         // 128-token blocks per statistics item
+
+enum QuantScheme : int { kSchemeI8Block = 0, kSchemeI8Token = 1, kSchemeNvfp4 = 2 };
+enum QuantItemKind : int { kItemKStat = 0, kItemVStat = 1, kItemQ = 2, kItemK = 3, kItemV = 4, kItemEnd = 5 };
+
+// A queue item, or (in a stage slot) one tile of it: blocks blk .. blk +
+// nsub - 1 of one tensor of head bh; a slot holds block blk, its `rows`, and
+// its index `sub` within the item.
+struct QuantItem {
+  int kind, bh, blk, rows, sub, nsub;
+};
+
+struct QuantArgs {
+  const void *q, *k, *v;
+  uint8_t *q8, *k8, *vt8;      // codes
+  uint8_t *sq, *sk, *sv;       // scales: float32 (I8QK_F8PV) or E4M3 blocks (NVFP4)
+  float *mu;
+  double *ksum;
+  unsigned *vmax;
+  unsigned *done;              // [BH] statistics publications per head
+  unsigned *ticket;            // next ticket
+  int BH, N, nblk, nv;
+};
+
+// Statistics items per head: K (and, I8QK_F8PV, V) in groups of kStatBlocks blocks.
+__host__ __device__ __forceinline__ int quant_stat_items(int scheme, int nblk) {
+  const int groups = (nblk + kStatBlocks - 1) / kStatBlocks;
+  return scheme == kSchemeNvfp4 ? groups : 2 * groups;
+}
+
+// Number of items in the queue.
+__host__ __device__ __forceinline__ long long quant_items(int scheme, int BH, int nblk) {
+  return static_cast<long long>(BH) * (quant_stat_items(scheme, nblk) + 3 * nblk);
+}
+
+// Ticket -> item, in the order given in the file comment.
+__host__ __device__ __forceinline__ QuantItem quant_item(int scheme, unsigned t, int BH, int nblk, int N) {
+  const int nstat = quant_stat_items(scheme, nblk);
+  const unsigned a = static_cast<unsigned>(nstat + nblk);   // |A(h)|
+  const unsigned b = static_cast<unsigned>(2 * nblk);       // |B(h)|
+  QuantItem it;
+  it.kind = kItemEnd;
+  it.bh = it.blk = it.rows = it.sub = 0;
+  it.nsub = 1;
+  if (static_cast<long long>(t) >= quant_items(scheme, BH, nblk)) return it;
+  int h;
+  unsigned r;
+  bool in_a;
+  if (t < a) {
+    h = 0;
+    r = t;
+    in_a = true;
+  } else {
+    const unsigned p = (t - a) / (a + b);
+    const unsigned rr = (t - a) % (a + b);
+    if (p + 1 < static_cast<unsigned>(BH) && rr < a) {
+      h = static_cast<int>(p) + 1;
+      r = rr;
+      in_a = true;
+    } else {
+      h = static_cast<int>(p);
+      r = p + 1 < static_cast<unsigned>(BH) ? rr - a : rr;
+      in_a = false;
+    }
+  }
+  if (in_a) {
+    if (r < static_cast<unsigned>(nstat)) {
+      const int g = scheme == kSchemeNvfp4 ? static_cast<int>(r) : static_cast<int>(r >> 1);
+      it.kind = (scheme != kSchemeNvfp4 && (r & 1u)) ? kItemVStat : kItemKStat;
+      it.blk = g * kStatBlocks;
+      it.nsub = nblk - it.blk < kStatBlocks ? nblk - it.blk : kStatBlocks;
+    } else {
+      it.kind = kItemQ;
+      it.blk = static_cast<int>(r) - nstat;
+    }
+  } else {
+    it.kind = r < static_cast<unsigned>(nblk) ? kItemK : kItemV;
+    it.blk = static_cast<int>(r % static_cast<unsigned>(nblk));
+  }
+  it.bh = h;
+  it.rows = N - it.blk * kBlockTokens < kBlockTokens ? N - it.blk * kBlockTokens : kBlockTokens;
+  return it;
+}
+
+template <int D>
+struct QuantSmem {
+  static constexpr int kTileBytes = kBlockTokens * D * 2;
+  static constexpr int kTiles = 0;
+  static constexpr int kChan = kTiles + kQuantStages * kTileBytes;     // per stage: mu or s_v [D]
+  static constexpr int kScratch = kChan + kQuantStages * D * 4;
+  static constexpr int kSlots = kScratch + ((static_cast<int>(sizeof(QuantScratch<D>)) + 15) / 16) * 16;
+  static constexpr int kBars = kSlots + ((kQuantStages * static_cast<int>(sizeof(QuantItem)) + 7) / 8) * 8;
+  static constexpr int kFlags = kBars + 2 * kQuantStages * 8;
+  static constexpr int kBytes = kFlags + 16;
+  static constexpr int kAlloc = kBytes + 128;      // room to align the base to 128 bytes
+};
+
+// Bounded spin of one thread until *count >= target (acquire at GPU scope).
+__device__ __forceinline__ bool wait_count(const unsigned *count, unsigned target, volatile int *abort_flag) {
+  if (ld_acquire_gpu(count) >= target) return true;
+  const long long t0 = clock64();
+  while (ld_acquire_gpu(count) < target) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > g_wait_limit) {
+      atomicOr(&g_error_word, kErrWaitTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(100);
+  }
+  return true;
+}
+
+// The compute warps' work on one tile.
+template <typename T, int D, int SCHEME>
+__device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &it, const T *tile, const float *cs,
+                                           QuantScratch<D> &sc, uint64_t *empty) {
+  constexpr bool NV = SCHEME == kSchemeNvfp4;
+  const size_t hrow = static_cast<size_t>(it.bh) * a.N;   // first row of the head
+  const int tok0 = it.blk * kBlockTokens;
+  const size_t sblk = static_cast<size_t>(it.bh) * a.nblk + it.blk;
+  switch (it.kind) {
+    case kItemKStat:
+      stat_tile<T, D, false>(tile, it.rows, it.sub == 0, sc, empty);
+      if (it.sub == it.nsub - 1)
+        stat_publish<D, false>(sc, a.ksum + static_cast<size_t>(it.bh) * D, nullptr, a.done + it.bh);
+      break;
+    case kItemVStat:
+      stat_tile<T, D, true>(tile, it.rows, it.sub == 0, sc, empty);
+      if (it.sub == it.nsub - 1)
+        stat_publish<D, true>(sc, nullptr, a.vmax + static_cast<size_t>(it.bh) * D, a.done + it.bh);
+      break;
+    case kItemQ:
+      if (NV)
+        nvfp4_rows_tile<T, D, false>(tile, it.rows, cs, a.q8 + (hrow + tok0) * (D / 2), a.sq + sblk * (D / 64) * 512,
+                                     empty);
+      else if (SCHEME == kSchemeI8Token)
+        q_token_tile<T, D>(tile, it.rows, sc, reinterpret_cast<int8_t *>(a.q8) + (hrow + tok0) * D,
+                           reinterpret_cast<float *>(a.sq) + hrow + tok0, empty);
+      else
+        qk_block_tile<T, D, false>(tile, it.rows, cs, sc, reinterpret_cast<int8_t *>(a.q8) + (hrow + tok0) * D,
+                                   reinterpret_cast<float *>(a.sq) + sblk, empty);
+      break;
+    case kItemK:
+      if (NV)
+        nvfp4_rows_tile<T, D, true>(tile, it.rows, cs, a.k8 + (hrow + tok0) * (D / 2), a.sk + sblk * (D / 64) * 512,
+                                    empty);
+      else
+        qk_block_tile<T, D, true>(tile, it.rows, cs, sc, reinterpret_cast<int8_t *>(a.k8) + (hrow + tok0) * D,
+                                  reinterpret_cast<float *>(a.sk) + sblk, empty);
+      break;
+    default:   // kItemV
+      if (NV)
+        nvfp4_v_tile<T, D>(tile, it.rows, tok0, a.nv, a.vt8 + static_cast<size_t>(it.bh) * D * (a.nv / 2),
+                           a.sv + sblk * 1024, empty);
+      else
+        v_tile<T, D>(tile, it.rows, tok0, a.nv, cs, a.vt8 + static_cast<size_t>(it.bh) * D * a.nv, empty);
+      break;
+  }
+}
+
+template <typename T, int D, int SCHEME>
+__global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs a) {
+  using L = QuantSmem<D>;
+  constexpr bool NV = SCHEME == kSchemeNvfp4;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  QuantScratch<D> &sc = *reinterpret_cast<QuantScratch<D> *>(smem + L::kScratch);
+  float *chan = reinterpret_cast<float *>(smem + L::kChan);
+  QuantItem *slot = reinterpret_cast<QuantItem *>(smem + L::kSlots);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBars);
+  uint64_t *empty = full + kQuantStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlags);
+  volatile int *go = abort_flag + 1;               // go[0], go[1]: per-tile decision of thread 0
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQuantStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kQuantWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (threadIdx.x >= kQuantConsumers) {
+    // ------------------------------------------------------------ producer warp
+    // Lane 0 takes tickets (one ahead, so that the atomic's latency overlaps
+    // the item's copies) and issues one copy per tile of the item; for a K or
+    // V tile the whole warp then waits for the head's statistics and writes
+    // the stage's per-channel mu (K) or s_v (V), before the stage's `full`
+    // barrier is arrived on: the compute warps find everything in shared
+    // memory.
+    const int lane = threadIdx.x & 31;
+    // every statistics item is published once per warp that issued accumulator atomics
+    const unsigned stats_target = static_cast<unsigned>(quant_stat_items(SCHEME, a.nblk)) * (D / 32);
+    uint64_t keep = 0, stream = 0;
+    unsigned next = 0;
+    if (lane == 0) {
+      keep = make_l2_policy_evict_last();
+      stream = make_l2_policy_evict_first();
+      next = atomicAdd(a.ticket, 1u);
+    }
+    int i = 0;                                     // stage uses issued
+    bool stop = false;
+    while (!stop) {
+      const QuantItem item = quant_item(SCHEME, __shfl_sync(0xffffffffu, next, 0), a.BH, a.nblk, a.N);
+      if (lane == 0 && item.kind != kItemEnd) next = atomicAdd(a.ticket, 1u);
+      for (int sub = 0; sub < item.nsub; ++sub) {
+        const int s = i % kQuantStages;
+        bool ok = true;
+        if (lane == 0 && i >= kQuantStages) ok = mbar_wait(&empty[s], ((i / kQuantStages) - 1) & 1, abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        QuantItem it = item;
+        it.blk = item.blk + sub;
+        it.sub = sub;
+        it.rows = a.N - it.blk * kBlockTokens < kBlockTokens ? a.N - it.blk * kBlockTokens : kBlockTokens;
+        if (it.kind == kItemEnd) {
+          if (lane == 0) {
+            slot[s] = it;
+            mbar_arrive(&full[s]);
+          }
+          ++i;
+          stop = true;
+          break;
+        }
+        if (lane == 0) {
+          slot[s] = it;
+          const void *base = (it.kind == kItemQ) ? a.q : (it.kind == kItemK || it.kind == kItemKStat) ? a.k : a.v;
+          const T *src = static_cast<const T *>(base) +
+                         (static_cast<size_t>(it.bh) * a.N + static_cast<size_t>(it.blk) * kBlockTokens) * D;
+          const uint32_t bytes = static_cast<uint32_t>(it.rows) * D * sizeof(T);
+          mbar_expect_tx(&full[s], bytes);
+          bulk_load(smem + L::kTiles + s * L::kTileBytes, src, bytes, &full[s],
+                    (it.kind == kItemKStat || it.kind == kItemVStat) ? keep : stream);
+        }
+        if (it.kind == kItemK || (!NV && it.kind == kItemV)) {
+          bool ready = true;
+          if (lane == 0) ready = wait_count(a.done + it.bh, stats_target, abort_flag);
+          if (__shfl_sync(0xffffffffu, ready, 0)) {
+            float *cs = chan + s * D;
+#pragma unroll
+            for (int c = lane; c < D; c += 32) {
+              const size_t hc = static_cast<size_t>(it.bh) * D + c;
+              if (it.kind == kItemK) {
+                const float mu = static_cast<float>(__ldcg(a.ksum + hc) / static_cast<double>(a.N));
+                cs[c] = mu;
+                if (it.blk == 0) a.mu[hc] = mu;
+              } else {
+                const float m = __uint_as_float(__ldcg(a.vmax + hc));
+                const float sv = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+                cs[c] = sv;
+                if (it.blk == 0) reinterpret_cast<float *>(a.sv)[hc] = sv;
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);      // release: the slot and the stage's channel values
+        ++i;
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
+          stop = true;
+          break;
+        }
+      }
+    }
+    // every copy this warp issued lands before the CTA can exit
+    if (lane == 0)
+      for (int u = i > kQuantStages ? i - kQuantStages : 0; u < i; ++u)
+        drain_wait(&full[u % kQuantStages], (u / kQuantStages) & 1);
+    return;
+  }
+
+  // -------------------------------------------------------------- compute warps
+  const int ct = threadIdx.x;
+  for (int i = 0;; ++i) {
+    const int s = i % kQuantStages;
+    const uint32_t par = (i / kQuantStages) & 1;
+    if (ct == 0) {
+      bool ok = mbar_wait(&full[s], par, abort_flag) && !*abort_flag;
+      if (ok && slot[s].kind == kItemEnd) ok = false;
+      go[i & 1] = ok ? 1 : 0;
+    }
+    __syncwarp();
+    named_bar_sync(kQuantBar, kQuantConsumers);
+    if (!go[i & 1]) break;
+    mbar_try_wait(&full[s], par);                  // completed: orders this thread after the copy
+    const QuantItem it = slot[s];
+    quant_tile<T, D, SCHEME>(a, it, reinterpret_cast<const T *>(smem + L::kTiles + s * L::kTileBytes), chan + s * D,
+                             sc, &empty[s]);
+  }
+}
+
+}  // namespace sattn

@@ -1,13 +1,14 @@
-// Quantisation kernels of the INT8-QK / FP8-PV mode.
+// Quantisation of the INT8-QK / FP8-PV mode: the per-tile work of the fused
+// quantiser (quant_fused.cuh schedules it).
 //
 // The TurboDiffusion explainer (wxsanhe.com post 64219, section 1 "hybrid
 // attention") puts QK^T in INT8 and PV in FP8 and recovers accuracy with
 // outlier smoothing; the SageAttention tag page (reportify.cn), SageAttention3
 // summary, bullet [17], quantises Q/K per block.  Readings used here:
-//   mu[c]   = (float)( sum_n K[n,c] (exact float64 sum) / N )      per (b,h)
+//   mu[c]   = (float)( sum_n K[n,c] (float64 sum) / N )      per (b,h)
 //   s_q, s_k = max|x| / 127 per 128-token block (1 for an all-zero block);
 //             optionally s_q per token (max over the token's channels)
-//   q8      = RNE(x / s) clamped to [-127, 127], division in IEEE float32
+//   q8      = RNE(x / s) clamped to [-127, 127], x / s the IEEE float32 quotient
 //   s_v[c]  = max_n |V[n,c]| / 448 per channel (1 for an all-zero channel)
 //   v8      = E4M3_RNE_satfinite(V / s_v), written transposed [d, Nv]
 //
@@ -15,48 +16,63 @@
 // the scale it feeds NaN: a Q block's (or token's) rows, a K channel's mean
 // (and with it every K scale of the head), a V channel's scale.
 //
-// HBM-bound.  Pass 1 (kv_stats) reads K and V once and reduces per-channel
-// sums in float64 atomics and per-channel |V| maxima.  Each bf16/fp16 value is
-// exact in float64, and so is every partial sum while the sum's magnitude
-// stays below 2^53 times the smallest quantum among the summands (true for
-// the workloads here: values above 2^-30 in magnitude, sums below 2^21), so
-// the mean does not depend on the order of the atomics; a head holding values
-// as small as fp16/bf16 subnormals next to sums near 2^30 can differ in the
-// mean's last bit between runs.  Pass 2 reads Q, K, V once more and writes
-// the codes; every load is a coalesced 16-byte vector.
+// A "tile" is 128 tokens x d channels of one tensor of one (b,h), staged in
+// shared memory row-major by a bulk copy; rows at and past `rows` are stale
+// and never read as data.  The 256 compute threads of a CTA take part in each
+// tile; every warp arrives once on the stage's `empty` barrier after its last
+// read of the tile.
+//
+// Statistics tiles add float64 column sums of K and float32 column maxima of
+// |V| into per-head accumulators with atomics.  Each bf16/fp16 value is exact
+// in float64, and so is every partial sum while the sum's magnitude stays
+// below 2^53 times the smallest quantum among the summands (true for the
+// workloads here: values above 2^-30 in magnitude, sums below 2^21), so the
+// mean does not depend on the order of the atomics; a head holding values as
+// small as fp16/bf16 subnormals next to sums near 2^30 can differ in the
+// mean's last bit between runs.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace sattn {
 
-constexpr int kBlockTokens = 128;   // quantisation block = attention tile height
-constexpr int kQuantThreads = 256;
-// Threads of the per-block quantizers: a block of 128 tokens is spread over
-// 512 threads so that each holds few values and an SM keeps more loads in flight.
-constexpr int kBlockQuantThreads = 512;
+constexpr int kBlockTokens = 128;      // quantisation block = attention tile height
+constexpr int kQuantConsumers = 256;   // compute threads of a quantiser CTA (8 warps)
+constexpr int kQuantWarps = kQuantConsumers / 32;
+constexpr int kQuantBar = 1;           // named barrier of the compute threads
 
+// Shared scratch of the compute threads.
+template <int D>
+struct QuantScratch {
+  union {
+    double sum[kQuantWarps][D];        // per-warp partial column sums of a K tile
+    float max[kQuantWarps][D];         // per-warp partial column maxima of a V tile
+  } red;
+  float red_max[kQuantWarps];          // per-warp maxima of a quantisation block
+  float row_scale[kBlockTokens];       // per-token Q scales of the tile (its rare exact path)
+};
+
+// 8 values (one 16-byte word) -> float, exact.
 template <typename T>
-__device__ __forceinline__ void load8(const T *p, float (&f)[8]);
+__device__ __forceinline__ void cvt8(const uint4 &u, float (&f)[8]);
 
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+__device__ __forceinline__ void cvt8<__nv_bfloat16>(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
 
 template <>
-__device__ __forceinline__ void load8<__half>(const __half *p, float (&f)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+__device__ __forceinline__ void cvt8<__half>(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -66,270 +82,476 @@ __device__ __forceinline__ void load8<__half>(const __half *p, float (&f)[8]) {
   }
 }
 
-// Pass 1: per-channel float64 sums of K and float32 maxima of |V|.
-// grid (ceil(N / tokens_per_cta), B*H), block 256.
+// Value i (0..7) of one 16-byte word of T -> float, exact.
+template <typename T>
+__device__ __forceinline__ float elem8(const uint4 &u, int i) {
+  const uint32_t w = i < 2 ? u.x : i < 4 ? u.y : i < 6 ? u.z : u.w;
+  if (std::is_same<T, __nv_bfloat16>::value) return __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+  const __half2 h = *reinterpret_cast<const __half2 *>(&w);
+  return (i & 1) ? __high2float(h) : __low2float(h);
+}
+
+// 8 consecutive values of a shared-memory tile (16-byte aligned) -> float.
+template <typename T>
+__device__ __forceinline__ void lds8(const T *p, float (&f)[8]) {
+  cvt8<T>(*reinterpret_cast<const uint4 *>(p), f);
+}
+
+// Lane-wise operations on two packed values of T (exact: maxima and minima
+// of representable values are representable), NaN-propagating.
+template <typename T>
+struct Packed;
+template <>
+struct Packed<__nv_bfloat16> {
+  using P = __nv_bfloat162;
+  static constexpr uint32_t kNegInf = 0xFF80FF80u, kPosInf = 0x7F807F80u;
+};
+template <>
+struct Packed<__half> {
+  using P = __half2;
+  static constexpr uint32_t kNegInf = 0xFC00FC00u, kPosInf = 0x7C007C00u;
+};
+template <typename T>
+__device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {   // max(acc, |w|)
+  using P = typename Packed<T>::P;
+  const P r = __hmax2_nan(*reinterpret_cast<const P *>(&acc), __habs2(*reinterpret_cast<const P *>(&w)));
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+template <typename T>
+__device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {
+  using P = typename Packed<T>::P;
+  const P r = __hmax2_nan(*reinterpret_cast<const P *>(&a), *reinterpret_cast<const P *>(&b));
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+template <typename T>
+__device__ __forceinline__ uint32_t min2(uint32_t a, uint32_t b) {
+  using P = typename Packed<T>::P;
+  const P r = __hmin2_nan(*reinterpret_cast<const P *>(&a), *reinterpret_cast<const P *>(&b));
+  return *reinterpret_cast<const uint32_t *>(&r);
+}
+// Both values of a packed pair as floats.
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+  const uint4 u = make_uint4(w, 0u, 0u, 0u);
+  return make_float2(elem8<T>(u, 0), elem8<T>(u, 1));
+}
+
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ void release_stage(uint64_t *empty) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
+}
+
+// This thread's rows of a tile, loaded into registers before any arithmetic
+// (so that the rows can be processed with full instruction-level
+// parallelism): row r0 + p (256 / (d/8)), channels 8 cg .. + 7, zeros for
+// rows at and past `rows`.
 template <typename T, int D>
-__global__ void __launch_bounds__(kQuantThreads) kv_stats_kernel(const T *__restrict__ k, const T *__restrict__ v,
-                                                                 double *__restrict__ ksum,
-                                                                 unsigned *__restrict__ vmax, int N,
-                                                                 int tokens_per_cta) {
-  constexpr int LPR = D / 8;                  // threads per row (8 channels each)
-  constexpr int RPI = kQuantThreads / LPR;    // rows per iteration
-  __shared__ double s_sum[RPI][D];
-  __shared__ float s_max[RPI][D];
+constexpr int kRowPasses = kBlockTokens * D / (8 * kQuantConsumers);
 
-  const int bh = blockIdx.y;
-  const int cg = threadIdx.x % LPR;
-  const int r0 = threadIdx.x / LPR;
-  const int n_begin = blockIdx.x * tokens_per_cta;
-  const int n_end = min(N, n_begin + tokens_per_cta);
-  const size_t head = static_cast<size_t>(bh) * N * D;
-
-  double acc[8];
-  float vm[8];
+template <typename T, int D>
+__device__ __forceinline__ void load_rows(const T *tile, int rows, int r0, int cg, uint4 (&u)[kRowPasses<T, D>]) {
+  constexpr int RPP = kQuantConsumers / (D / 8);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    acc[i] = 0.0;
-    vm[i] = 0.f;
-  }
-#pragma unroll 4
-  for (int n = n_begin + r0; n < n_end; n += RPI) {
-    float kf[8], vf[8];
-    load8<T>(k + head + static_cast<size_t>(n) * D + cg * 8, kf);
-    load8<T>(v + head + static_cast<size_t>(n) * D + cg * 8, vf);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      acc[i] += static_cast<double>(kf[i]);
-      vm[i] = fmax_nan(vm[i], fabsf(vf[i]));
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    s_sum[r0][cg * 8 + i] = acc[i];
-    s_max[r0][cg * 8 + i] = vm[i];
-  }
-  __syncthreads();
-  if (threadIdx.x < D) {
-    const int c = threadIdx.x;
-    double s = 0.0;
-    float m = 0.f;
-    for (int r = 0; r < RPI; ++r) {
-      s += s_sum[r][c];
-      m = fmax_nan(m, s_max[r][c]);
-    }
-    atomicAdd(ksum + static_cast<size_t>(bh) * D + c, s);
-    atomicMax(vmax + static_cast<size_t>(bh) * D + c, __float_as_uint(m));  // m >= 0: bit order = value order
+  for (int p = 0; p < kRowPasses<T, D>; ++p) {
+    const int r = r0 + p * RPP;
+    u[p] = r < rows ? *reinterpret_cast<const uint4 *>(tile + r * D + cg * 8) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
-template <int NT>
-__device__ __forceinline__ float block_max(float v, float *s_red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int warp = threadIdx.x >> 5;
-  if ((threadIdx.x & 31) == 0) s_red[warp] = v;
-  __syncthreads();
-  float m = s_red[0];
-#pragma unroll
-  for (int w = 1; w < NT / 32; ++w) m = fmax_nan(m, s_red[w]);
-  return m;
-}
-
-// Pass 2a: per-block INT8 of Q (IS_K = false) or of K - mu (IS_K = true).
-// grid (ceil(N/128), B*H), block kBlockQuantThreads.  Each thread owns a
-// fixed group of 8 channels and (128 * D / 8) / kBlockQuantThreads row positions.
-template <typename T, int D, bool IS_K>
-__global__ void __launch_bounds__(kBlockQuantThreads, 2) quant_qk_kernel(const T *__restrict__ x, int8_t *__restrict__ out,
-                                                                 float *__restrict__ scale,
-                                                                 const double *__restrict__ ksum,
-                                                                 float *__restrict__ mu_out, int N, int nblk) {
+// One tile of a statistics item (several consecutive 128-token blocks of one
+// tensor of one head): per-channel sums of K (IS_V = false) or maxima of |V|
+// (IS_V = true) over the tile's rows (zero rows past `rows` change neither),
+// reduced within each warp and kept per warp in sc.red (first = the item's
+// first tile: overwrite, else accumulate).  Thread ct takes the 8 channels
+// 8 (ct mod d/8) .. + 7 of every (256 / (d/8))-th row; each (warp, channel)
+// slot has one writer.
+template <typename T, int D, bool IS_V>
+__device__ __forceinline__ void stat_tile(const T *tile, int rows, bool first, QuantScratch<D> &sc,
+                                          uint64_t *empty) {
   constexpr int LPR = D / 8;
-  constexpr int RPI = kBlockQuantThreads / LPR;
-  constexpr int ITERS = kBlockTokens / RPI;
-  __shared__ float s_red[kBlockQuantThreads / 32];
-
-  const int bh = blockIdx.y;
-  const int blk = blockIdx.x;
-  const int cg = threadIdx.x % LPR;
-  const int r0 = threadIdx.x / LPR;
-  const size_t head = static_cast<size_t>(bh) * N * D;
-
-  // every load first, so that the mean's float64 division below overlaps them
-  float val[ITERS][8];
+  constexpr int PASSES = kRowPasses<T, D>;
+  const int ct = threadIdx.x;
+  const int lane = ct & 31;
+  const int warp = ct >> 5;
+  const int cg = ct % LPR;
+  uint4 u[PASSES];
+  load_rows<T, D>(tile, rows, ct / LPR, cg, u);
+  release_stage(empty);
+  if (IS_V) {
+    uint32_t vm[4] = {0u, 0u, 0u, 0u};             // packed max |V| of the 8 channels
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int n = blk * kBlockTokens + it * RPI + r0;
-    if (n < N) {
-      load8<T>(x + head + static_cast<size_t>(n) * D + cg * 8, val[it]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) val[it][i] = 0.f;
+    for (int p = 0; p < PASSES; ++p) {
+      vm[0] = absmax2<T>(vm[0], u[p].x);
+      vm[1] = absmax2<T>(vm[1], u[p].y);
+      vm[2] = absmax2<T>(vm[2], u[p].z);
+      vm[3] = absmax2<T>(vm[3], u[p].w);
     }
-  }
-  float amax = 0.f;
-  if (IS_K) {
-    float mu[8];
+    float m[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      mu[i] = static_cast<float>(ksum[static_cast<size_t>(bh) * D + cg * 8 + i] / static_cast<double>(N));
-    if (blk == 0 && r0 == 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mu_out[static_cast<size_t>(bh) * D + cg * 8 + i] = mu[i];
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = unpack2<T>(vm[i]);
+      m[2 * i] = t.x;
+      m[2 * i + 1] = t.y;
     }
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const bool valid = blk * kBlockTokens + it * RPI + r0 < N;
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = fmax_nan(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+    if (lane < LPR) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        val[it][i] = valid ? __fsub_rn(val[it][i], mu[i]) : 0.f;
-        amax = fmax_nan(amax, fabsf(val[it][i]));
+        float &slot = sc.red.max[warp][cg * 8 + i];
+        slot = first ? m[i] : fmax_nan(slot, m[i]);
       }
     }
   } else {
+    double acc[8];
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it)
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmax_nan(amax, fabsf(val[it][i]));
-  }
-  amax = block_max<kBlockQuantThreads>(amax, s_red);
-  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
-  if (threadIdx.x == 0) scale[static_cast<size_t>(bh) * nblk + blk] = s;
-
+    for (int p = 0; p < PASSES; ++p) {
+      float f[8];
+      cvt8<T>(u[p], f);
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int n = blk * kBlockTokens + it * RPI + r0;
-    if (n < N) {
-      uint32_t w[2] = {0u, 0u};
+      for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(f[i]);
+    }
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (lane < LPR) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        int qi = __float2int_rn(__fdiv_rn(val[it][i], s));
-        qi = max(-127, min(127, qi));
-        w[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
+        double &slot = sc.red.sum[warp][cg * 8 + i];
+        slot = first ? acc[i] : slot + acc[i];
       }
-      *reinterpret_cast<uint2 *>(out + head + static_cast<size_t>(n) * D + cg * 8) = make_uint2(w[0], w[1]);
     }
   }
 }
 
-// Pass 2a, per-token variant: INT8 of Q with one scale per token ("thread-level"
-// granularity: the attention kernel gives each query row its own thread), s =
-// max|x[n, :]| / 127.  grid (ceil(N / kTokRows), B*H), block kQuantThreads;
-// D/8 consecutive lanes share a token (8 channels each) and every thread takes
-// kTokIters tokens, loaded before any is reduced.
-constexpr int kTokIters = 4;
-template <int D>
-__host__ __device__ constexpr int tok_rows_per_cta() { return kQuantThreads / (D / 8) * kTokIters; }
-
-template <typename T, int D>
-__global__ void __launch_bounds__(kQuantThreads) quant_q_token_kernel(const T *__restrict__ x, int8_t *__restrict__ out,
-                                                                      float *__restrict__ scale, int N) {
-  constexpr int LPR = D / 8;                  // lanes per token (16 or 8); divides 32
-  constexpr int RPI = kQuantThreads / LPR;    // tokens per iteration of the CTA
-  const int bh = blockIdx.y;
-  const int cg = threadIdx.x % LPR;
-  const size_t head = static_cast<size_t>(bh) * N * D;
-  const int n0 = blockIdx.x * tok_rows_per_cta<D>() + threadIdx.x / LPR;
-  float val[kTokIters][8];
+// End of a statistics item: the per-warp slots are summed (maximised) over
+// the CTA and added into the head's accumulator (ksum_h or vmax_h, d
+// entries) by threads ct < d; each of their warps then fences its atomics
+// and bumps *done_h once (a warp-level publication: no barrier across warps).
+template <int D, bool IS_V>
+__device__ __forceinline__ void stat_publish(QuantScratch<D> &sc, double *ksum_h, unsigned *vmax_h,
+                                             unsigned *done_h) {
+  const int ct = threadIdx.x;
+  named_bar_sync(kQuantBar, kQuantConsumers);
+  if (ct < D) {
+    if (IS_V) {
+      float m = sc.red.max[0][ct];
 #pragma unroll
-  for (int it = 0; it < kTokIters; ++it) {
-    const int n = n0 + it * RPI;
-    if (n < N) {
-      load8<T>(x + head + static_cast<size_t>(n) * D + cg * 8, val[it]);
+      for (int w = 1; w < kQuantWarps; ++w) m = fmax_nan(m, sc.red.max[w][ct]);
+      atomicMax(vmax_h + ct, __float_as_uint(m));   // m >= 0 or NaN: bit order = value order
     } else {
+      double s = sc.red.sum[0][ct];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) val[it][i] = 0.f;
+      for (int w = 1; w < kQuantWarps; ++w) s += sc.red.sum[w][ct];
+      atomicAdd(ksum_h + ct, s);
+    }
+    __threadfence();
+    __syncwarp();                                   // d is a multiple of 32: whole warps
+    if ((ct & 31) == 0) {
+      __threadfence();
+      atomicAdd(done_h, 1u);
+    }
+  }
+}
+
+// INT8 codes RNE(x / s) (s > 0 finite, r = 1/s correctly rounded, the IEEE
+// float32 quotient being the reference) of 8 values, packed lowest index in
+// the lowest byte, by the product x * r: for |x / s| <= 128, x * r lies within
+// 2.5e-5 of the exact quotient and the IEEE quotient within 7.7e-6, so both
+// round to the same integer unless x * r is within 1e-4 of a half-integer.
+// Returns false in that case (the caller then takes int8_codes8_exact).  The
+// rounding adds 1.5 * 2^23, which puts RNE(y) in the low mantissa bits (exact
+// for |y| < 2^22): the code byte is the low byte of the sum's bit pattern.
+__device__ __forceinline__ bool int8_codes8_fast(const float (&x)[8], float r, uint2 &codes) {
+  constexpr float kRound = 12582912.0f;            // 1.5 * 2^23
+  const float2 r2 = make_float2(r, r);
+  const float2 k2 = make_float2(kRound, kRound);
+  const float2 m1 = make_float2(-1.f, -1.f);
+  uint32_t c[8];
+  float worst = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 y = fmul2(make_float2(x[2 * j], x[2 * j + 1]), r2);
+    const float2 m = fadd2(y, k2);
+    const float2 t = fadd2(y, ffma2(m, m1, k2));  // y - RNE(y), exact
+    worst = fmax3(worst, fabsf(t.x), fabsf(t.y));
+    c[2 * j] = __float_as_uint(m.x);
+    c[2 * j + 1] = __float_as_uint(m.y);
+  }
+  codes = make_uint2(__byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410),
+                     __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410));
+  return worst <= 0.4999f;
+}
+
+// The same codes through the IEEE quotient (near ties, and scales whose
+// reciprocal is not a positive normal number); a NaN quotient gives code 0.
+__device__ __forceinline__ uint2 int8_codes8_exact(const float (&x)[8], float s) {
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int qi = __float2int_rn(__fdiv_rn(x[i], s));
+    qi = max(-127, min(127, qi));
+    w[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ bool fast_reciprocal(float r) { return r > 0.f && r < 3.0e38f; }
+
+// Per-block INT8 of a Q tile (IS_K = false) or of K - mu (IS_K = true, mu =
+// the stage's per-channel values): one scale for the tile's valid rows, codes
+// into out_blk (row r at out_blk + r d), the scale into *scale_slot.  The
+// block maximum is taken on the packed inputs: max |x| for Q, and for K
+// max(RN(max x - mu), RN(mu - min x)) per channel, which equals the maximum
+// of |RN(x - mu)| because rounding is monotone.
+template <typename T, int D, bool IS_K>
+__device__ __forceinline__ void qk_block_tile(const T *tile, int rows, const float *mu_s, QuantScratch<D> &sc,
+                                              int8_t *out_blk, float *scale_slot, uint64_t *empty) {
+  constexpr int LPR = D / 8;
+  constexpr int RPP = kQuantConsumers / LPR;
+  constexpr int PASSES = kRowPasses<T, D>;
+  const int ct = threadIdx.x;
+  const int lane = ct & 31;
+  const int warp = ct >> 5;
+  const int cg = ct % LPR;
+  const int r0 = ct / LPR;
+  float nmu[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) nmu[i] = IS_K ? -mu_s[cg * 8 + i] : 0.f;
+  uint4 u[PASSES];
+  load_rows<T, D>(tile, rows, r0, cg, u);
+
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hi[i] = IS_K ? Packed<T>::kNegInf : 0u;
+    lo[i] = Packed<T>::kPosInf;
+  }
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const bool valid = r0 + p * RPP < rows;        // a zero row is not data for the K extrema
+    const uint32_t w[4] = {u[p].x, u[p].y, u[p].z, u[p].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (IS_K) {
+        hi[i] = max2<T>(hi[i], valid ? w[i] : Packed<T>::kNegInf);
+        lo[i] = min2<T>(lo[i], valid ? w[i] : Packed<T>::kPosInf);
+      } else {
+        hi[i] = absmax2<T>(hi[i], w[i]);
+      }
+    }
+  }
+  float amax = 0.f;
+  if (!IS_K || r0 < rows) {                        // no rows: no term (mu may be infinite)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 h = unpack2<T>(hi[i]);
+      if (IS_K) {
+        const float2 l = unpack2<T>(lo[i]);
+        amax = fmax3_nan(amax, __fadd_rn(h.x, nmu[2 * i]), __fsub_rn(-nmu[2 * i], l.x));
+        amax = fmax3_nan(amax, __fadd_rn(h.y, nmu[2 * i + 1]), __fsub_rn(-nmu[2 * i + 1], l.y));
+      } else {
+        amax = fmax3_nan(amax, h.x, h.y);
+      }
     }
   }
 #pragma unroll
-  for (int it = 0; it < kTokIters; ++it) {
-    const int n = n0 + it * RPI;
-    float amax = 0.f;
+  for (int o = 16; o > 0; o >>= 1) amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) sc.red_max[warp] = amax;
+  named_bar_sync(kQuantBar, kQuantConsumers);
+  amax = sc.red_max[0];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmax_nan(amax, fabsf(val[it][i]));
-    // every lane of the warp takes part (tokens past N hold zeros)
+  for (int w = 1; w < kQuantWarps; ++w) amax = fmax_nan(amax, sc.red_max[w]);
+  const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  const float rcp = __frcp_rn(s);
+  if (ct == 0) *scale_slot = s;
+
+  unsigned redo = fast_reciprocal(rcp) ? 0u : (1u << PASSES) - 1u;
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    float f[8];
+    cvt8<T>(u[p], f);
+    if (IS_K) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 d = fadd2(make_float2(f[2 * j], f[2 * j + 1]), make_float2(nmu[2 * j], nmu[2 * j + 1]));
+        f[2 * j] = d.x;
+        f[2 * j + 1] = d.y;
+      }
+    }
+    uint2 codes;
+    if (!int8_codes8_fast(f, rcp, codes)) redo |= 1u << p;
+    const int r = r0 + p * RPP;
+    if (r < rows) *reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8) = codes;
+  }
+  // rare: rows near a rounding tie again, through the IEEE quotient (from the stage)
+  for (; redo != 0u; redo &= redo - 1u) {
+    const int r = r0 + (__ffs(redo) - 1) * RPP;
+    if (r >= rows) continue;
+    float f[8];
+    lds8<T>(tile + r * D + cg * 8, f);
+    if (IS_K) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = __fadd_rn(f[i], nmu[i]);
+    }
+    *reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8) = int8_codes8_exact(f, s);
+  }
+  release_stage(empty);
+}
+
+// Per-token INT8 of a Q tile ("thread-level" granularity: the attention
+// kernel gives each query row its own thread): s = max|x[n, :]| / 127 for
+// every valid row, into scale_blk[r].  The d/8 lanes of a row reduce its
+// maximum with shuffles; every lane takes part (rows past `rows` hold zeros).
+template <typename T, int D>
+__device__ __forceinline__ void q_token_tile(const T *tile, int rows, QuantScratch<D> &sc, int8_t *out_blk,
+                                             float *scale_blk, uint64_t *empty) {
+  constexpr int LPR = D / 8;
+  constexpr int RPP = kQuantConsumers / LPR;
+  constexpr int PASSES = kRowPasses<T, D>;
+  const int ct = threadIdx.x;
+  const int cg = ct % LPR;
+  const int r0 = ct / LPR;
+  uint4 u[PASSES];
+  load_rows<T, D>(tile, rows, r0, cg, u);
+  unsigned redo = 0u;
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const float2 mf = unpack2<T>(absmax2<T>(absmax2<T>(absmax2<T>(absmax2<T>(0u, u[p].x), u[p].y), u[p].z), u[p].w));
+    float amax = fmax_nan(mf.x, mf.y);
 #pragma unroll
     for (int o = LPR / 2; o > 0; o >>= 1) amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float s = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
-    if (n < N) {
-      if (cg == 0) scale[static_cast<size_t>(bh) * N + n] = s;
-      uint32_t w[2] = {0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        int qi = __float2int_rn(__fdiv_rn(val[it][i], s));
-        qi = max(-127, min(127, qi));
-        w[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
-      }
-      *reinterpret_cast<uint2 *>(out + head + static_cast<size_t>(n) * D + cg * 8) = make_uint2(w[0], w[1]);
+    const float rcp = __frcp_rn(s);
+    float f[8];
+    cvt8<T>(u[p], f);
+    uint2 codes;
+    if (!int8_codes8_fast(f, rcp, codes) || !fast_reciprocal(rcp)) redo |= 1u << p;
+    const int r = r0 + p * RPP;
+    if (cg == 0) sc.row_scale[r] = s;
+    if (r < rows) {
+      if (cg == 0) scale_blk[r] = s;
+      *reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8) = codes;
     }
   }
+  __syncwarp();                                    // a row's lanes share a warp: its scale is visible
+  // rare: rows near a rounding tie again, through the IEEE quotient (from the stage)
+  for (; redo != 0u; redo &= redo - 1u) {
+    const int r = r0 + (__ffs(redo) - 1) * RPP;
+    if (r >= rows) continue;
+    float f[8];
+    lds8<T>(tile + r * D + cg * 8, f);
+    *reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8) = int8_codes8_exact(f, sc.row_scale[r]);
+  }
+  release_stage(empty);
 }
 
-// Pass 2b: per-channel FP8 E4M3 of V, stored transposed vt[bh][c][token]
-// with row length Nv (N rounded up to 16).  grid (ceil(N/128), B*H), block
-// 4 D threads.  Thread t takes the 4 tokens 4 (t mod 32) .. + 3 of the block
-// and the 8 channels of group t / 32, packs the 4 codes of each channel into one word
-// (lowest token in the low byte), and the block is written out row by row:
-// every shared-memory access of a warp touches 32 consecutive words and every
-// global store is a full 128-byte row segment.
+// The bracket multipliers of a divisor: rlo = RN(r (1 - 2^-20)), rhi =
+// RN(r (1 + 2^-20)), r = RN(1/sv).  For any x, the products x rlo and x rhi
+// bracket both the exact quotient x / sv and its float32 rounding (their
+// relative error is below 2^-22), and rounding to a narrower format is
+// monotone: when the two ends give the same code, that is the quotient's
+// code.  False when r is not a positive normal number below 1e38.
+__device__ __forceinline__ bool bracket(float sv, float &rlo, float &rhi) {
+  const float r = __frcp_rn(sv);
+  rlo = r * 0.99999904632568359375f;               // 1 - 2^-20
+  rhi = r * 1.00000095367431640625f;               // 1 + 2^-20
+  return r > 1.2e-38f && r < 1.0e38f;
+}
+
+// E4M3 codes of 4 values of one channel by the bracket; returns the codes of
+// the upper end and clears `ok` when the ends disagree.
+__device__ __forceinline__ uint32_t e4m3_codes4_fast(const float (&x)[4], float rlo, float rhi, bool &ok) {
+  const float2 a = make_float2(x[0], x[1]);
+  const float2 b = make_float2(x[2], x[3]);
+  const float2 alo = fmul2(a, make_float2(rlo, rlo));
+  const float2 blo = fmul2(b, make_float2(rlo, rlo));
+  const float2 ahi = fmul2(a, make_float2(rhi, rhi));
+  const float2 bhi = fmul2(b, make_float2(rhi, rhi));
+  const uint32_t clo = cvt_e4m3x2(alo.x, alo.y) | (cvt_e4m3x2(blo.x, blo.y) << 16);
+  const uint32_t chi = cvt_e4m3x2(ahi.x, ahi.y) | (cvt_e4m3x2(bhi.x, bhi.y) << 16);
+  ok = ok && clo == chi;
+  return chi;
+}
+
+template <int G>
+__device__ __forceinline__ void store_codes(uint8_t *dst, const uint32_t (&w)[G]) {
+  if (G == 2)
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[G - 1]);
+  else
+    *reinterpret_cast<uint32_t *>(dst) = w[0];
+}
+
+// Per-channel FP8 E4M3 of a V tile (s_v = the stage's per-channel values),
+// written transposed into vt_h[c * Nv + tok0 + t] for the tile's tokens below
+// Nv (tokens at and past N get code 0).  Warp w takes 4 TPT tokens of 64
+// channels; lane l the 8 channels 8 (l mod 8) .. + 7 of that half and the TPT
+// tokens TPT (l / 8) ..; it packs the TPT codes of each channel (lowest token
+// in the lowest byte) and stores them with one vector store, so that the four
+// lanes of a channel write 4 TPT consecutive bytes.
 template <typename T, int D>
-__global__ void __launch_bounds__(4 * D, 2) quant_v_kernel(const T *__restrict__ v, uint8_t *__restrict__ vt,
-                                                                float *__restrict__ sv_out,
-                                                                const unsigned *__restrict__ vmax, int N,
-                                                                int Nv) {
-  constexpr int CPT = 8;                     // channels per thread
-  constexpr int NT = 4 * D;                  // threads
-  constexpr int WPR = kBlockTokens / 4;      // words per channel row of the block (32)
-  __shared__ uint32_t tile[D][WPR];
-
-  const int bh = blockIdx.y;
-  const int blk = blockIdx.x;
-  const int tq = threadIdx.x % WPR;          // token quad
-  const int c0 = (threadIdx.x / WPR) * CPT;  // first channel of this thread
-  const size_t head = static_cast<size_t>(bh) * N * D;
-
-  float sv[CPT];
+__device__ __forceinline__ void v_tile(const T *tile, int rows, int tok0, int Nv, const float *sv_s, uint8_t *vt_h,
+                                       uint64_t *empty) {
+  constexpr int TPT = D == 128 ? 8 : 4;            // tokens per thread
+  constexpr int TPW = 4 * TPT;                     // tokens per warp
+  constexpr int WPT = kBlockTokens / TPW;          // warps along the tokens
+  constexpr int G = TPT / 4;                       // 4-token groups per thread
+  static_assert(WPT * (D / 64) == kQuantWarps, "one V task per warp");
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int c0 = (warp / WPT) * 64 + (lane % 8) * 8;
+  const int t0 = (warp % WPT) * TPW + (lane / 8) * TPT;
+  uint4 raw[TPT];                                  // the tokens' 8 channels, unconverted (zeros past `rows`)
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const float m = __uint_as_float(vmax[static_cast<size_t>(bh) * D + c0 + i]);
-    sv[i] = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
-  }
-  if (blk == 0 && tq == 0) {
+  for (int t = 0; t < TPT; ++t)
+    raw[t] = t0 + t < rows ? *reinterpret_cast<const uint4 *>(tile + (t0 + t) * D + c0) : make_uint4(0u, 0u, 0u, 0u);
+  unsigned redo = 0u;
+  if (tok0 + t0 < Nv) {                            // Nv is a multiple of 16: all TPT tokens in or out
 #pragma unroll
-    for (int i = 0; i < CPT; ++i) sv_out[static_cast<size_t>(bh) * D + c0 + i] = sv[i];
-  }
-
-  float f[4][CPT];
+    for (int i = 0; i < 8; ++i) {
+      float rlo, rhi;
+      bool ok = bracket(sv_s[c0 + i], rlo, rhi);
+      uint32_t w[G];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int n = blk * kBlockTokens + 4 * tq + r;
-#pragma unroll
-    for (int g = 0; g < CPT; g += 8) {
-      float t8[8];
-      if (n < N) {
-        load8<T>(v + head + static_cast<size_t>(n) * D + c0 + g, t8);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) t8[i] = 0.f;
+      for (int g = 0; g < G; ++g) {
+        const float x[4] = {elem8<T>(raw[4 * g], i), elem8<T>(raw[4 * g + 1], i), elem8<T>(raw[4 * g + 2], i),
+                            elem8<T>(raw[4 * g + 3], i)};
+        w[g] = e4m3_codes4_fast(x, rlo, rhi, ok);
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) f[r][g + i] = t8[i];
+      if (!ok) redo |= 1u << i;
+      store_codes<G>(vt_h + static_cast<size_t>(c0 + i) * Nv + tok0 + t0, w);
     }
   }
+  // rare: channels with a code near a rounding boundary again, through the
+  // IEEE quotient (values from the stage)
+  for (; redo != 0u; redo &= redo - 1u) {
+    const int c = c0 + __ffs(redo) - 1;
+    const float sv = sv_s[c];
+    uint32_t w[G];
 #pragma unroll
-  for (int i = 0; i < CPT; ++i) {
-    const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f[0][i], sv[i]), __fdiv_rn(f[1][i], sv[i]));
-    const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f[2][i], sv[i]), __fdiv_rn(f[3][i], sv[i]));
-    tile[c0 + i][tq] = lo | (hi << 16);
+    for (int g = 0; g < G; ++g) {
+      float q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = t0 + 4 * g + j;
+        q[j] = t < rows ? __fdiv_rn(static_cast<float>(tile[t * D + c]), sv) : 0.f;
+      }
+      w[g] = cvt_e4m3x2(q[0], q[1]) | (cvt_e4m3x2(q[2], q[3]) << 16);
+    }
+    store_codes<G>(vt_h + static_cast<size_t>(c) * Nv + tok0 + t0, w);
   }
-  __syncthreads();
-  const int tok0 = blk * kBlockTokens;
-  const int valid_words = min(kBlockTokens, Nv - tok0) / 4;
-  for (int idx = threadIdx.x; idx < D * WPR; idx += NT) {
-    const int c = idx / WPR;
-    const int w = idx % WPR;
-    if (w < valid_words)
-      *reinterpret_cast<uint32_t *>(vt + (static_cast<size_t>(bh) * D + c) * Nv + tok0 + 4 * w) = tile[c][w];
-  }
+  release_stage(empty);
 }
 
 }  // namespace sattn

@@ -1,4 +1,5 @@
-// Quantisation kernels of the NVFP4 mode.
+// Quantisation of the NVFP4 mode: the per-tile work of the fused quantiser
+// (quant_fused.cuh schedules it).
 //
 // SageAttention tag page (reportify.cn), SageAttention3 summary, FP4 bullet
 // [15]: microscaled FP4 with the NVFP4 format -- E2M1 values, one E4M3 scale
@@ -51,8 +52,9 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
 }
 
 // One NVFP4 block of 16 values: returns the E4M3 scale code and writes the 8
-// code bytes (as two 32-bit words).
-__device__ __forceinline__ uint32_t nvfp4_block(const float (&x)[16], uint32_t (&w)[2]) {
+// code bytes (as two 32-bit words), E2M1(x / scale) through the IEEE
+// quotient.  A block whose scale rounds to 0 (or is NaN) gets zero codes.
+__device__ __forceinline__ uint32_t nvfp4_block_exact(const float (&x)[16], uint32_t (&w)[2]) {
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmax_nan(amax, fabsf(x[i]));
@@ -69,98 +71,166 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float (&x)[16], uint32_t (
   return sc_code;
 }
 
-// Q (IS_K = false) or K - mu (IS_K = true): one thread per (row, 16-channel
-// block).  grid (ceil(N/128), B*H), block 256.
-template <typename T, int D, bool IS_K>
-__global__ void __launch_bounds__(kQuantThreads) quant_rows_nvfp4_kernel(const T *__restrict__ x,
-                                                                         uint8_t *__restrict__ codes,
-                                                                         uint8_t *__restrict__ sf,
-                                                                         const double *__restrict__ ksum,
-                                                                         float *__restrict__ mu_out, int N) {
-  constexpr int BPR = D / 16;                      // blocks per row
-  constexpr int SF_TILE = (D / 64) * 512;          // scale bytes per 128-row tile
-  __shared__ float s_mu[D];
-  const int bh = blockIdx.y;
-  const int tile = blockIdx.x;
-  const size_t head = static_cast<size_t>(bh) * N * D;
-  const int ntiles = gridDim.x;
-  if (IS_K) {
-    if (threadIdx.x < D) {
-      const float mu = static_cast<float>(ksum[static_cast<size_t>(bh) * D + threadIdx.x] / static_cast<double>(N));
-      s_mu[threadIdx.x] = mu;
-      if (tile == 0) mu_out[static_cast<size_t>(bh) * D + threadIdx.x] = mu;
+// The same block with the codes by the bracket of `bracket` (x RN(r (1 -+
+// 2^-20)), r = RN(1/scale)): E2M1 rounding is monotone, so equal codes at
+// both ends are the quotient's codes.  Clears `ok` when they differ (the
+// caller then takes nvfp4_block_exact).
+__device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&x)[16], uint32_t (&w)[2], bool &ok) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmax_nan(amax, fabsf(x[i]));
+  const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
+  const float sc = e4m3_to_float(sc_code);
+  w[0] = w[1] = 0u;
+  if (sc > 0.f) {
+    float rlo, rhi;
+    ok = bracket(sc, rlo, rhi) && ok;
+    uint32_t lo[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 pl = fmul2(make_float2(x[i], x[i + 1]), make_float2(rlo, rlo));
+      const float2 ph = fmul2(make_float2(x[i], x[i + 1]), make_float2(rhi, rhi));
+      lo[i >> 3] |= cvt_e2m1x2(pl.x, pl.y) << (4 * (i & 7));
+      w[i >> 3] |= cvt_e2m1x2(ph.x, ph.y) << (4 * (i & 7));
     }
-    __syncthreads();
+    ok = ok && lo[0] == w[0] && lo[1] == w[1];
   }
-  uint8_t *sf_tile = sf + (static_cast<size_t>(bh) * ntiles + tile) * SF_TILE;
-  for (int idx = threadIdx.x; idx < kBlockTokens * BPR; idx += kQuantThreads) {
-    const int r = idx / BPR;
-    const int b = idx % BPR;
-    const int n = tile * kBlockTokens + r;
-    float v[16];
-    if (n < N) {
-      float a[8], c[8];
-      load8<T>(x + head + static_cast<size_t>(n) * D + b * 16, a);
-      load8<T>(x + head + static_cast<size_t>(n) * D + b * 16 + 8, c);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[i] = a[i];
-        v[8 + i] = c[i];
-      }
-      if (IS_K) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], s_mu[b * 16 + i]);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = 0.f;
-    }
-    uint32_t w[2];
-    const uint32_t sc = nvfp4_block(v, w);
-    if (n < N) *reinterpret_cast<uint2 *>(codes + (head + static_cast<size_t>(n) * D) / 2 + b * 8) = make_uint2(w[0], w[1]);
-    sf_tile[(b >> 2) * 512 + sf_offset(r, b)] = static_cast<uint8_t>(sc);
-  }
+  return sc_code;
 }
 
-// V: blocks of 16 tokens of one channel, written transposed vt[bh][c][Nv/2].
-// grid (ceil(N/128), B*H), block 256.
-template <typename T, int D>
-__global__ void __launch_bounds__(kQuantThreads) quant_v_nvfp4_kernel(const T *__restrict__ v, uint8_t *__restrict__ vt,
-                                                                      uint8_t *__restrict__ sf, int N, int Nv) {
-  __shared__ T tile_v[kBlockTokens][D + 2];
-  const int bh = blockIdx.y;
-  const int tile = blockIdx.x;
-  const size_t head = static_cast<size_t>(bh) * N * D;
-  const int ntiles = gridDim.x;
-  for (int idx = threadIdx.x; idx < kBlockTokens * D / 8; idx += kQuantThreads) {
-    const int r = idx / (D / 8);
-    const int cg = idx % (D / 8);
-    const int n = tile * kBlockTokens + r;
-    float a[8];
-    if (n < N) {
-      load8<T>(v + head + static_cast<size_t>(n) * D + cg * 8, a);
-    } else {
+// NVFP4 of a Q tile (IS_K = false) or of K - mu (IS_K = true, mu = the
+// stage's per-channel values): thread ct takes the 16-channel block ct mod
+// (d/16) of every (256 / (d/16))-th row.  Codes of valid rows into codes_blk
+// (row r at codes_blk + r d/2); the scale of every row (0 for rows past
+// `rows`) into the tile's scale-factor blocks sf_tile.
+template <typename T, int D, bool IS_K>
+__device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const float *mu_s, uint8_t *codes_blk,
+                                                uint8_t *sf_tile, uint64_t *empty) {
+  constexpr int BPR = D / 16;                      // blocks per row
+  constexpr int RPP = kQuantConsumers / BPR;
+  constexpr int PASSES = kBlockTokens / RPP;
+  const int ct = threadIdx.x;
+  const int b = ct % BPR;
+  const int r0 = ct / BPR;
+  float mu[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = 0.f;
+  for (int i = 0; i < 16; ++i) mu[i] = IS_K ? mu_s[b * 16 + i] : 0.f;
+  uint4 u[PASSES][2];                              // every row first
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int r = r0 + p * RPP;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      u[p][h] = r < rows ? *reinterpret_cast<const uint4 *>(tile + r * D + b * 16 + 8 * h) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  unsigned redo = 0u;
+#pragma unroll
+  for (int p = 0; p < PASSES; ++p) {
+    const int r = r0 + p * RPP;
+    float v[16];
+    float a[8], c[8];
+    cvt8<T>(u[p][0], a);
+    cvt8<T>(u[p][1], c);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = a[i];
+      v[8 + i] = c[i];
     }
+    if (IS_K && r < rows) {                        // rows past `rows` stay zero
 #pragma unroll
-    for (int i = 0; i < 8; ++i) tile_v[r][cg * 8 + i] = static_cast<T>(a[i]);
-  }
-  __syncthreads();
-  uint8_t *sf_tile = sf + (static_cast<size_t>(bh) * ntiles + tile) * 1024;
-  for (int idx = threadIdx.x; idx < D * (kBlockTokens / 16); idx += kQuantThreads) {
-    const int c = idx % D;
-    const int t = idx / D;                         // 16-token block within the tile
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = static_cast<float>(tile_v[t * 16 + i][c]);
+      for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], mu[i]);
+    }
     uint32_t w[2];
-    const uint32_t sc = nvfp4_block(x, w);
-    const int tok0 = tile * kBlockTokens + t * 16;
-    if (tok0 < Nv)
-      *reinterpret_cast<uint2 *>(vt + (static_cast<size_t>(bh) * D + c) * (Nv / 2) + tok0 / 2) = make_uint2(w[0], w[1]);
-    sf_tile[(t >> 2) * 512 + sf_offset(c, t)] = static_cast<uint8_t>(sc);
+    bool ok = true;
+    const uint32_t sc_code = nvfp4_block_fast(v, w, ok);
+    if (!ok) redo |= 1u << p;
+    if (r < rows) *reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8) = make_uint2(w[0], w[1]);
+    sf_tile[(b >> 2) * 512 + sf_offset(r, b)] = static_cast<uint8_t>(sc_code);
   }
+  // rare: blocks near a rounding boundary again, through the IEEE quotient (from the stage)
+  for (; redo != 0u; redo &= redo - 1u) {
+    const int r = r0 + (__ffs(redo) - 1) * RPP;
+    if (r >= rows) continue;
+    float v[16];
+    float a[8], c[8];
+    lds8<T>(tile + r * D + b * 16, a);
+    lds8<T>(tile + r * D + b * 16 + 8, c);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = IS_K ? __fsub_rn(a[i], mu[i]) : a[i];
+      v[8 + i] = IS_K ? __fsub_rn(c[i], mu[8 + i]) : c[i];
+    }
+    uint32_t w[2];
+    nvfp4_block_exact(v, w);
+    *reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8) = make_uint2(w[0], w[1]);
+  }
+  release_stage(empty);
+}
+
+// NVFP4 of a V tile: blocks of 16 tokens of one channel, written transposed
+// into vt_h[c * Nv/2 + (tok0 + t)/2] for tokens below Nv (tokens at and past
+// N are zeros).  Warp w < 4 d/64 takes 32 tokens of 64 channels; lane l the
+// channel pair 2 l, 2 l + 1 of that half, read as one 32-bit word per token
+// (a warp reads 128 consecutive bytes of a row), and stores 16 code bytes
+// per channel.
+template <typename T, int D>
+__device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, int Nv, uint8_t *vt_h,
+                                             uint8_t *sf_tile, uint64_t *empty) {
+  constexpr int NCH = D / 64;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  if (warp < 4 * NCH) {
+    const int tg = warp / NCH;                     // 32-token group of the tile
+    const int c = 2 * ((warp % NCH) * 32 + lane);  // first channel of the pair
+    float x[2][32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      const int r = tg * 32 + t;
+      const uint32_t u = r < rows ? *reinterpret_cast<const uint32_t *>(tile + r * D + c) : 0u;
+      const float2 f = unpack2<T>(u);
+      x[0][t] = f.x;
+      x[1][t] = f.y;
+    }
+    unsigned redo = 0u;
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float blk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) blk[i] = x[ch][16 * h + i];
+        uint32_t wh[2];
+        bool ok = true;
+        const uint32_t sc_code = nvfp4_block_fast(blk, wh, ok);
+        if (!ok) redo |= 1u << (2 * ch + h);
+        w[2 * h] = wh[0];
+        w[2 * h + 1] = wh[1];
+        const int t16 = 2 * tg + h;                // 16-token block of the tile
+        sf_tile[(t16 >> 2) * 512 + sf_offset(c + ch, t16)] = static_cast<uint8_t>(sc_code);
+      }
+      if (tok0 + tg * 32 < Nv)                     // Nv is a multiple of 32
+        *reinterpret_cast<uint4 *>(vt_h + static_cast<size_t>(c + ch) * (Nv / 2) + (tok0 + tg * 32) / 2) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    // rare: blocks near a rounding boundary again, through the IEEE quotient (from the stage)
+    for (; redo != 0u; redo &= redo - 1u) {
+      const int k = __ffs(redo) - 1;
+      const int ch = k >> 1, h = k & 1;
+      float blk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = tg * 32 + 16 * h + i;
+        blk[i] = r < rows ? static_cast<float>(tile[r * D + c + ch]) : 0.f;
+      }
+      uint32_t wh[2];
+      nvfp4_block_exact(blk, wh);
+      if (tok0 + tg * 32 < Nv)
+        *reinterpret_cast<uint2 *>(vt_h + static_cast<size_t>(c + ch) * (Nv / 2) + (tok0 + tg * 32 + 16 * h) / 2) =
+            make_uint2(wh[0], wh[1]);
+    }
+  }
+  release_stage(empty);
 }
 
 }  // namespace sattn

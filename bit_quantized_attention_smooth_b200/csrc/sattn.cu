@@ -14,8 +14,7 @@
 #include "../../include/sattn.h"
 #include "attn_i8f8.cuh"
 #include "attn_nvfp4.cuh"
-#include "quant_i8f8.cuh"
-#include "quant_nvfp4.cuh"
+#include "quant_fused.cuh"
 
 namespace sattn {
 namespace {
@@ -53,6 +52,10 @@ bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr
 
 bool is_nvfp4(int mode) { return base_mode(mode) == SATTN_NVFP4; }
 
+// The vmax section holds vmax[BH][d] and then the quantiser's work counters:
+// done[BH] and the ticket counter.  Offset of done from the section start.
+size_t counters_offset(size_t BH, int d) { return BH * d * sizeof(unsigned); }
+
 // NVFP4 workspace: q8/k8/vt8 hold the packed E2M1 codes of Q, K - mean and
 // V^T (N rounded up to 32 tokens), sq/sk/sv the E4M3 scale blocks of Q, K, V.
 sattn_ws_layout_t make_layout_nvfp4(int B, int H, int N, int d) {
@@ -70,7 +73,7 @@ sattn_ws_layout_t make_layout_nvfp4(int B, int H, int N, int d) {
   L.sv = off;   off = align_up(off + BH * L.nblk * 1024, kSectionAlign);
   L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.ksum = off; off += BH * d * sizeof(double);
-  L.vmax = off; off = align_up(off + BH * d * sizeof(unsigned), kSectionAlign);
+  L.vmax = off; off = align_up(off + counters_offset(BH, d) + (BH + 1) * sizeof(unsigned), kSectionAlign);
   L.total = off;
   return L;
 }
@@ -92,7 +95,7 @@ sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d, bool per_token) {
   L.sv = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.ksum = off; off += BH * d * sizeof(double);
-  L.vmax = off; off = align_up(off + BH * d * sizeof(unsigned), kSectionAlign);
+  L.vmax = off; off = align_up(off + counters_offset(BH, d) + (BH + 1) * sizeof(unsigned), kSectionAlign);
   L.total = off;
   return L;
 }
@@ -154,51 +157,52 @@ bool make_map_u8(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int D>
-int launch_quant_i8f8(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws,
-                      const sattn_ws_layout_t &L, bool per_token, cudaStream_t st) {
-  double *ksum = reinterpret_cast<double *>(ws + L.ksum);
-  unsigned *vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
-  if (cudaMemsetAsync(ws + L.ksum, 0, L.total - L.ksum, st) != cudaSuccess) return SATTN_ERR_CUDA;
-  const int tpc = 512;
-  kv_stats_kernel<T, D><<<dim3((N + tpc - 1) / tpc, BH), kQuantThreads, 0, st>>>(
-      static_cast<const T *>(k), static_cast<const T *>(v), ksum, vmax, N, tpc);
-  const dim3 grid(L.nblk, BH);
-  if (per_token) {
-    const int rows = tok_rows_per_cta<D>();
-    quant_q_token_kernel<T, D><<<dim3((N + rows - 1) / rows, BH), kQuantThreads, 0, st>>>(
-        static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq), N);
-  } else {
-    quant_qk_kernel<T, D, false><<<grid, kBlockQuantThreads, 0, st>>>(
-        static_cast<const T *>(q), reinterpret_cast<int8_t *>(ws + L.q8), reinterpret_cast<float *>(ws + L.sq),
-        nullptr, nullptr, N, L.nblk);
-  }
-  quant_qk_kernel<T, D, true><<<grid, kBlockQuantThreads, 0, st>>>(
-      static_cast<const T *>(k), reinterpret_cast<int8_t *>(ws + L.k8), reinterpret_cast<float *>(ws + L.sk), ksum,
-      reinterpret_cast<float *>(ws + L.mu), N, L.nblk);
-  quant_v_kernel<T, D><<<grid, 4 * D, 0, st>>>(static_cast<const T *>(v), ws + L.vt8,
-                                                        reinterpret_cast<float *>(ws + L.sv), vmax, N, L.nv);
-  g_launches += 4;
-  return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+// SMs of the current device (persistent grids).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
 }
 
-template <typename T, int D>
-int launch_quant_nvfp4(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws,
-                       const sattn_ws_layout_t &L, cudaStream_t st) {
-  double *ksum = reinterpret_cast<double *>(ws + L.ksum);
-  unsigned *vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
+// The quantiser (quant_fused.cuh): zeroes the statistics accumulators and
+// work counters (and, NVFP4, the V scale blocks, whose rows past d are never
+// written), then one persistent launch of two CTAs per SM.
+template <typename T, int D, int SCHEME>
+int launch_quant(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws, const sattn_ws_layout_t &L,
+                 cudaStream_t st) {
   if (cudaMemsetAsync(ws + L.ksum, 0, L.total - L.ksum, st) != cudaSuccess) return SATTN_ERR_CUDA;
-  if (cudaMemsetAsync(ws + L.sv, 0, static_cast<size_t>(BH) * L.nblk * 1024, st) != cudaSuccess) return SATTN_ERR_CUDA;
-  const int tpc = 512;
-  kv_stats_kernel<T, D><<<dim3((N + tpc - 1) / tpc, BH), kQuantThreads, 0, st>>>(
-      static_cast<const T *>(k), static_cast<const T *>(v), ksum, vmax, N, tpc);
-  const dim3 grid(L.nblk, BH);
-  quant_rows_nvfp4_kernel<T, D, false><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(q), ws + L.q8, ws + L.sq,
-                                                                       nullptr, nullptr, N);
-  quant_rows_nvfp4_kernel<T, D, true><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(k), ws + L.k8, ws + L.sk,
-                                                                      ksum, reinterpret_cast<float *>(ws + L.mu), N);
-  quant_v_nvfp4_kernel<T, D><<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(v), ws + L.vt8, ws + L.sv, N, L.nv);
-  g_launches += 4;
+  if (SCHEME == kSchemeNvfp4 &&
+      cudaMemsetAsync(ws + L.sv, 0, static_cast<size_t>(BH) * L.nblk * 1024, st) != cudaSuccess)
+    return SATTN_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return SATTN_ERR_CUDA;
+  auto kern = quant_kernel<T, D, SCHEME>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QuantSmem<D>::kAlloc) != cudaSuccess)
+    return SATTN_ERR_CUDA;
+  QuantArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q8 = ws + L.q8;
+  a.k8 = ws + L.k8;
+  a.vt8 = ws + L.vt8;
+  a.sq = ws + L.sq;
+  a.sk = ws + L.sk;
+  a.sv = ws + L.sv;
+  a.mu = reinterpret_cast<float *>(ws + L.mu);
+  a.ksum = reinterpret_cast<double *>(ws + L.ksum);
+  a.vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
+  a.done = reinterpret_cast<unsigned *>(ws + L.vmax + counters_offset(BH, D));
+  a.ticket = a.done + BH;
+  a.BH = BH;
+  a.N = N;
+  a.nblk = L.nblk;
+  a.nv = L.nv;
+  const long long items = quant_items(SCHEME, BH, L.nblk);
+  const int grid = static_cast<int>(std::min<long long>(2LL * sms, items));
+  kern<<<grid, kQuantThreads, QuantSmem<D>::kAlloc, st>>>(a);
+  g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
@@ -363,17 +367,23 @@ int sattn_quantize(const void *q, const void *k, const void *v, int B, int H, in
   const bool fp16 = (mode & SATTN_FP16_IO) != 0;
   if (is_nvfp4(mode)) {
     if (d == 128)
-      return fp16 ? launch_quant_nvfp4<__half, 128>(q, k, v, BH, N, ws, L, cs)
-                  : launch_quant_nvfp4<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, cs);
-    return fp16 ? launch_quant_nvfp4<__half, 64>(q, k, v, BH, N, ws, L, cs)
-                : launch_quant_nvfp4<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, cs);
+      return fp16 ? launch_quant<__half, 128, kSchemeNvfp4>(q, k, v, BH, N, ws, L, cs)
+                  : launch_quant<__nv_bfloat16, 128, kSchemeNvfp4>(q, k, v, BH, N, ws, L, cs);
+    return fp16 ? launch_quant<__half, 64, kSchemeNvfp4>(q, k, v, BH, N, ws, L, cs)
+                : launch_quant<__nv_bfloat16, 64, kSchemeNvfp4>(q, k, v, BH, N, ws, L, cs);
   }
-  const bool pt = q_per_token(mode);
+  if (q_per_token(mode)) {
+    if (d == 128)
+      return fp16 ? launch_quant<__half, 128, kSchemeI8Token>(q, k, v, BH, N, ws, L, cs)
+                  : launch_quant<__nv_bfloat16, 128, kSchemeI8Token>(q, k, v, BH, N, ws, L, cs);
+    return fp16 ? launch_quant<__half, 64, kSchemeI8Token>(q, k, v, BH, N, ws, L, cs)
+                : launch_quant<__nv_bfloat16, 64, kSchemeI8Token>(q, k, v, BH, N, ws, L, cs);
+  }
   if (d == 128)
-    return fp16 ? launch_quant_i8f8<__half, 128>(q, k, v, BH, N, ws, L, pt, cs)
-                : launch_quant_i8f8<__nv_bfloat16, 128>(q, k, v, BH, N, ws, L, pt, cs);
-  return fp16 ? launch_quant_i8f8<__half, 64>(q, k, v, BH, N, ws, L, pt, cs)
-              : launch_quant_i8f8<__nv_bfloat16, 64>(q, k, v, BH, N, ws, L, pt, cs);
+    return fp16 ? launch_quant<__half, 128, kSchemeI8Block>(q, k, v, BH, N, ws, L, cs)
+                : launch_quant<__nv_bfloat16, 128, kSchemeI8Block>(q, k, v, BH, N, ws, L, cs);
+  return fp16 ? launch_quant<__half, 64, kSchemeI8Block>(q, k, v, BH, N, ws, L, cs)
+              : launch_quant<__nv_bfloat16, 64, kSchemeI8Block>(q, k, v, BH, N, ws, L, cs);
 }
 
 int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out, int B, int H, int N, int d, int causal,

@@ -97,7 +97,10 @@ size_t sattn_workspace_bytes(int B, int H, int N, int d, int mode);
  * (explainer, section 1: PV in FP8; V stored transposed, tokens contiguous).
  * NVFP4: E2M1 codes with one E4M3 scale per 16 values of Q, K - mean (along
  * channels) and V (along tokens) (tag page, bullet [15]).  A NaN input makes
- * the scale it feeds NaN.  Asynchronous on `stream`.  The workspace stays
+ * the scale it feeds NaN.  Asynchronous on `stream`: one memset of the
+ * workspace's scratch section and one kernel launch, whose tiles of K and V
+ * wait (bounded; on time-out the device error word records it, see
+ * sattn_device_error) for their head's statistics.  The workspace stays
  * valid for any number of sattn_fwd_quantized calls with the same
  * (B, H, N, d, mode).  Errors: see the header overview; nothing is written
  * when an argument is rejected. */
@@ -236,7 +239,8 @@ int sattn_device_error(int clear);
  *              vt8 e4m3   [B*H, d, Nv]  (Nv = N rounded up to 16)
  *              sq float32 [B*H, ceil(N/128)], or [B*H, N] with SATTN_Q_PER_TOKEN
  *              sk float32 [B*H, ceil(N/128)]   sv, mu float32 [B*H, d]
- *              ksum float64 [B*H, d], vmax uint32 [B*H, d] (scratch)
+ *              ksum float64 [B*H, d], vmax uint32 [B*H, d] followed by
+ *              the quantiser's work counters uint32 [B*H + 1] (scratch)
  *   NVFP4 (same fields, other contents):
  *              q8, k8 E2M1 codes, two per byte (low nibble = even channel)
  *                        [B*H, N, d/2]

@@ -63,7 +63,10 @@ QUANT_CASES = [W.SMALL,
 
 @pytest.mark.parametrize("w", QUANT_CASES, ids=lambda w: w.name)
 def test_quantizer_bit_exact(w):
-    q, k, v = W.make_inputs(w, "cuda")
+    _check_quantizer(w, *W.make_inputs(w, "cuda"))
+
+
+def _check_quantizer(w, q, k, v):
     ws = sattn.quantize(q, k, v)
     torch.cuda.synchronize()
     g = _ws_arrays(ws, w, q.dtype)
@@ -84,6 +87,46 @@ def test_quantizer_bit_exact(w):
             same = (gv == ov) | (((gv & 0x7F) == 0) & ((ov & 0x7F) == 0))
             assert same.all(), "V codes"
             assert np.array_equal(e4m3_decode(gv), e4m3_decode(ov))
+
+
+def _tie_inputs(w, seed):
+    """Inputs whose every code sits on a rounding tie of its format.
+
+    Every token of Q holds +-127 and every K token +-127 in channel 1, so all
+    INT8 scales (per block and per token) are exactly 1; the other Q and K
+    entries are n + 1/2.  K comes in +- pairs of tokens (a zero last token when
+    N is odd), so its channel means are exactly 0 and K - mean = K.  One V
+    token is 448 in every channel (s_v = 1) and the others are E4M3 midpoints,
+    normal and subnormal.  Each division is then exact and lands on a tie,
+    which RNE breaks to even: the kernels' reciprocal fast paths must fall
+    back to the IEEE quotient for every value."""
+    rng = np.random.default_rng(seed)
+    N, d = w.N, w.d
+    shape = (w.B, w.H, N, d)
+    q = rng.integers(-127, 127, size=shape) + 0.5
+    q[..., 0] = 127.0 * rng.choice([-1.0, 1.0], size=shape[:3])
+    half = rng.integers(-127, 127, size=(w.B, w.H, N // 2, d)) + 0.5
+    half[..., 1] = 127.0
+    k = np.zeros(shape)
+    k[:, :, 0:2 * (N // 2):2] = half
+    k[:, :, 1:2 * (N // 2):2] = -half
+    mids = [(1 + (2 * j + 1) / 16) * 2.0 ** e for e in range(-6, 8) for j in range(8)]
+    mids += [(m + 0.5) * 2.0 ** -9 for m in range(8)]
+    v = rng.choice(mids, size=shape) * rng.choice([-1.0, 1.0], size=shape)
+    v[:, :, rng.integers(0, N)] = 448.0
+    dt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+    t = [torch.tensor(x, dtype=torch.float64).to(dt) for x in (q, k, v)]
+    for a, x in zip(t, (q, k, v)):
+        assert np.array_equal(a.double().numpy(), x), "tie inputs must be exact in the I/O type"
+    return [a.cuda() for a in t]
+
+
+@pytest.mark.parametrize("w", [W.custom(1, 2, 300, 128, seed=61), W.custom(1, 1, 257, 64, "fp16", seed=62)],
+                         ids=lambda w: w.name)
+def test_quantizer_bit_exact_on_rounding_ties(w):
+    q, k, v = _tie_inputs(w, seed=w.seed)
+    _check_quantizer(w, q, k, v)
+    _check_per_token(w, q)
 
 
 OUTLIERS = "0.1 % of Q entries x20: per-{} INT8 Q carries the outliers' scale (emulation cosine {:.5f})"
@@ -139,8 +182,11 @@ def _check_attention(w, causal):
 @pytest.mark.parametrize("w", [W.custom(1, 2, 300, 128, seed=53, q_outlier_frac=1e-3),
                                W.custom(2, 1, 129, 64, "fp16", seed=54)], ids=lambda w: w.name)
 def test_per_token_q_quantizer_bit_exact(w):
-    q, k, v = W.make_inputs(w, "cuda")
-    ws = sattn.quantize(q, k, v, q_per_token=True)
+    _check_per_token(w, W.make_inputs(w, "cuda")[0])
+
+
+def _check_per_token(w, q):
+    ws = sattn.quantize(q, q, q, q_per_token=True)
     torch.cuda.synchronize()
     lay = sattn.workspace_layout(w.B, w.H, w.N, w.d, dtype=q.dtype, q_per_token=True)
     h = ws.cpu().numpy()

@@ -66,7 +66,43 @@ QUANT_CASES = [W.custom(1, 2, 256, 64, "fp16", seed=31),
 
 @pytest.mark.parametrize("w", QUANT_CASES, ids=lambda w: w.name)
 def test_nvfp4_quantizer_bit_exact(w):
-    q, k, v = W.make_inputs(w, "cuda")
+    _check_quantizer(w, *W.make_inputs(w, "cuda"))
+
+
+def _tie_inputs(w, seed):
+    """Inputs whose every FP4 code sits on an E2M1 rounding tie.
+
+    Every 16-value block (16 channels of a Q or K token, 16 tokens of a V
+    channel) holds a +-6, so its E4M3 scale is 6/6 = 1; the other values are
+    E2M1 midpoints.  K comes in +- pairs of tokens (a zero last token when N
+    is odd), so its channel means are exactly 0 and K - mean = K.  Each
+    division is then exact and lands on a tie, which RNE breaks to even: the
+    kernel's reciprocal fast path must fall back to the IEEE quotient."""
+    rng = np.random.default_rng(seed)
+    N, d = w.N, w.d
+    shape = (w.B, w.H, N, d)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    sign = lambda *sz: rng.choice([-1.0, 1.0], size=sz)
+    q = rng.choice(mids, size=shape) * sign(*shape)
+    q[..., 0::16] = 6.0 * sign(w.B, w.H, N, d // 16)
+    half = rng.choice(mids, size=(w.B, w.H, N // 2, d)) * sign(w.B, w.H, N // 2, d)
+    half[..., 0::16] = 6.0
+    k = np.zeros(shape)
+    k[:, :, 0:2 * (N // 2):2] = half
+    k[:, :, 1:2 * (N // 2):2] = -half
+    v = rng.choice(mids, size=shape) * sign(*shape)
+    v[:, :, 0::16] = 6.0 * sign(w.B, w.H, (N + 15) // 16, d)
+    dt = torch.float16 if w.dtype == "fp16" else torch.bfloat16
+    return [torch.tensor(x, dtype=torch.float64).to(dt).cuda() for x in (q, k, v)]
+
+
+@pytest.mark.parametrize("w", [W.custom(1, 2, 300, 128, seed=63), W.custom(1, 1, 257, 64, "fp16", seed=64)],
+                         ids=lambda w: w.name)
+def test_nvfp4_quantizer_bit_exact_on_rounding_ties(w):
+    _check_quantizer(w, *_tie_inputs(w, seed=w.seed))
+
+
+def _check_quantizer(w, q, k, v):
     ws = sattn.quantize(q, k, v, mode="nvfp4")
     torch.cuda.synchronize()
     lay = sattn.workspace_layout(w.B, w.H, w.N, w.d, mode="nvfp4", dtype=q.dtype)
