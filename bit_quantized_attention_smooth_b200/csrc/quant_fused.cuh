@@ -9,12 +9,14 @@
 //   B(h) = K tiles of h, then V tiles of h
 // A tile is 128 tokens x d of one tensor of one (b,h); a statistics item is
 // kStatBlocks consecutive tiles, reduced over the CTA and published once.
-// The order is A(0) A(1) B(0) A(2) B(1) ... A(BH-1) B(BH-2) B(BH-1): a head's
-// K and V are quantised about one head after their statistics were read, so
-// that their second read comes from L2 (two heads' K and V, about 34 MB at
-// N = 32760, d = 128, stay resident in the 126 MB L2; the statistics reads
-// carry an evict-last hint and every other read evict-first).  HBM then sees
-// each input byte once.
+// The order is A(0) .. A(L-1), then A(h+L) B(h) for h = 0, 1, ..: a head's K
+// and V are quantised L heads after their statistics were read, so that
+// their second read comes from L2 (the host picks L so that L + 1 heads' K
+// and V stay well inside the 126 MB L2, and so that the items taken but not
+// yet finished by all CTAs -- about four per CTA -- fit between a head's last
+// statistics item and its first K tile; the statistics reads carry an
+// evict-last hint and every other read evict-first).  HBM then sees each
+// input byte once.
 //
 // A K or V tile waits for its head's statistics: at the end of every
 // statistics item, each of the d/32 warps that add into the head's
@@ -41,7 +43,8 @@ namespace sattn {
 
 constexpr int kQuantStages = 3;
 constexpr int kQuantThreads = kQuantConsumers + 32;
-constexpr int kStatBlocks = 4;         // 128-token blocks per statistics item
+constexpr int kStatBlocks = 8;         // 128-token blocks per statistics item
+constexpr int kChanRows = 3;           // per-channel values a stage carries
 
 enum QuantScheme : int { kSchemeI8Block = 0, kSchemeI8Token = 1, kSchemeNvfp4 = 2 };
 enum QuantItemKind : int { kItemKStat = 0, kItemVStat = 1, kItemQ = 2, kItemK = 3, kItemV = 4, kItemEnd = 5 };
@@ -63,6 +66,7 @@ struct QuantArgs {
   unsigned *done;              // [BH] statistics publications per head
   unsigned *ticket;            // next ticket
   int BH, N, nblk, nv;
+  int lag;                     // heads whose statistics are read before B(0)
 };
 
 // Statistics items per head: K (and, I8QK_F8PV, V) in groups of kStatBlocks blocks.
@@ -76,11 +80,15 @@ __host__ __device__ __forceinline__ long long quant_items(int scheme, int BH, in
   return static_cast<long long>(BH) * (quant_stat_items(scheme, nblk) + 3 * nblk);
 }
 
-// Ticket -> item, in the order given in the file comment.
-__host__ __device__ __forceinline__ QuantItem quant_item(int scheme, unsigned t, int BH, int nblk, int N) {
+// Ticket -> item, in the order given in the file comment, with lag L =
+// min(lag, BH): A(0) .. A(L-1), then for h = 0 .. BH-1: A(h+L) (while h+L <
+// BH) followed by B(h).
+__host__ __device__ __forceinline__ QuantItem quant_item(int scheme, unsigned t, int BH, int nblk, int N, int lag) {
   const int nstat = quant_stat_items(scheme, nblk);
   const unsigned a = static_cast<unsigned>(nstat + nblk);   // |A(h)|
   const unsigned b = static_cast<unsigned>(2 * nblk);       // |B(h)|
+  const unsigned L = static_cast<unsigned>(lag < BH ? lag : BH);
+  const unsigned paired = static_cast<unsigned>(BH) - L;    // B(h) preceded by A(h+L)
   QuantItem it;
   it.kind = kItemEnd;
   it.bh = it.blk = it.rows = it.sub = 0;
@@ -89,22 +97,21 @@ __host__ __device__ __forceinline__ QuantItem quant_item(int scheme, unsigned t,
   int h;
   unsigned r;
   bool in_a;
-  if (t < a) {
-    h = 0;
-    r = t;
+  if (t < L * a) {
+    h = static_cast<int>(t / a);
+    r = t % a;
     in_a = true;
+  } else if (t - L * a < paired * (a + b)) {
+    const unsigned p = (t - L * a) / (a + b);
+    const unsigned rr = (t - L * a) % (a + b);
+    in_a = rr < a;
+    h = static_cast<int>(in_a ? p + L : p);
+    r = in_a ? rr : rr - a;
   } else {
-    const unsigned p = (t - a) / (a + b);
-    const unsigned rr = (t - a) % (a + b);
-    if (p + 1 < static_cast<unsigned>(BH) && rr < a) {
-      h = static_cast<int>(p) + 1;
-      r = rr;
-      in_a = true;
-    } else {
-      h = static_cast<int>(p);
-      r = p + 1 < static_cast<unsigned>(BH) ? rr - a : rr;
-      in_a = false;
-    }
+    const unsigned t3 = t - L * a - paired * (a + b);
+    h = static_cast<int>(paired + t3 / b);
+    r = t3 % b;
+    in_a = false;
   }
   if (in_a) {
     if (r < static_cast<unsigned>(nstat)) {
@@ -129,8 +136,10 @@ template <int D>
 struct QuantSmem {
   static constexpr int kTileBytes = kBlockTokens * D * 2;
   static constexpr int kTiles = 0;
-  static constexpr int kChan = kTiles + kQuantStages * kTileBytes;     // per stage: mu or s_v [D]
-  static constexpr int kScratch = kChan + kQuantStages * D * 4;
+  // per stage, kChanRows x D floats: mu (K tiles) or s_v, RN(r (1 - 2^-20)),
+  // RN(r (1 + 2^-20)) with r = RN(1/s_v) (V tiles)
+  static constexpr int kChan = kTiles + kQuantStages * kTileBytes;
+  static constexpr int kScratch = kChan + kQuantStages * kChanRows * D * 4;
   static constexpr int kSlots = kScratch + ((static_cast<int>(sizeof(QuantScratch<D>)) + 15) / 16) * 16;
   static constexpr int kBars = kSlots + ((kQuantStages * static_cast<int>(sizeof(QuantItem)) + 7) / 8) * 8;
   static constexpr int kFlags = kBars + 2 * kQuantStages * 8;
@@ -175,8 +184,8 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
       break;
     case kItemQ:
       if (NV)
-        nvfp4_rows_tile<T, D, false>(tile, it.rows, cs, a.q8 + (hrow + tok0) * (D / 2), a.sq + sblk * (D / 64) * 512,
-                                     empty);
+        nvfp4_rows_tile<T, D, false>(tile, it.rows, cs, sc.e4m3_recip, a.q8 + (hrow + tok0) * (D / 2),
+                                     a.sq + sblk * (D / 64) * 512, empty);
       else if (SCHEME == kSchemeI8Token)
         q_token_tile<T, D>(tile, it.rows, sc, reinterpret_cast<int8_t *>(a.q8) + (hrow + tok0) * D,
                            reinterpret_cast<float *>(a.sq) + hrow + tok0, empty);
@@ -186,16 +195,16 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
       break;
     case kItemK:
       if (NV)
-        nvfp4_rows_tile<T, D, true>(tile, it.rows, cs, a.k8 + (hrow + tok0) * (D / 2), a.sk + sblk * (D / 64) * 512,
-                                    empty);
+        nvfp4_rows_tile<T, D, true>(tile, it.rows, cs, sc.e4m3_recip, a.k8 + (hrow + tok0) * (D / 2),
+                                    a.sk + sblk * (D / 64) * 512, empty);
       else
         qk_block_tile<T, D, true>(tile, it.rows, cs, sc, reinterpret_cast<int8_t *>(a.k8) + (hrow + tok0) * D,
                                   reinterpret_cast<float *>(a.sk) + sblk, empty);
       break;
     default:   // kItemV
       if (NV)
-        nvfp4_v_tile<T, D>(tile, it.rows, tok0, a.nv, a.vt8 + static_cast<size_t>(it.bh) * D * (a.nv / 2),
-                           a.sv + sblk * 1024, empty);
+        nvfp4_v_tile<T, D>(tile, it.rows, tok0, a.nv, sc.e4m3_recip,
+                           a.vt8 + static_cast<size_t>(it.bh) * D * (a.nv / 2), a.sv + sblk * 1024, empty);
       else
         v_tile<T, D>(tile, it.rows, tok0, a.nv, cs, a.vt8 + static_cast<size_t>(it.bh) * D * a.nv, empty);
       break;
@@ -224,6 +233,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (NV) fill_e4m3_recip(sc.e4m3_recip);
   __syncthreads();
 
   if (threadIdx.x >= kQuantConsumers) {
@@ -247,7 +257,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
     int i = 0;                                     // stage uses issued
     bool stop = false;
     while (!stop) {
-      const QuantItem item = quant_item(SCHEME, __shfl_sync(0xffffffffu, next, 0), a.BH, a.nblk, a.N);
+      const QuantItem item = quant_item(SCHEME, __shfl_sync(0xffffffffu, next, 0), a.BH, a.nblk, a.N, a.lag);
       if (lane == 0 && item.kind != kItemEnd) next = atomicAdd(a.ticket, 1u);
       for (int sub = 0; sub < item.nsub; ++sub) {
         const int s = i % kQuantStages;
@@ -284,7 +294,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
           bool ready = true;
           if (lane == 0) ready = wait_count(a.done + it.bh, stats_target, abort_flag);
           if (__shfl_sync(0xffffffffu, ready, 0)) {
-            float *cs = chan + s * D;
+            float *cs = chan + s * kChanRows * D;
 #pragma unroll
             for (int c = lane; c < D; c += 32) {
               const size_t hc = static_cast<size_t>(it.bh) * D + c;
@@ -295,7 +305,11 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
               } else {
                 const float m = __uint_as_float(__ldcg(a.vmax + hc));
                 const float sv = m == 0.f ? 1.f : __fdiv_rn(m, 448.f);
+                float rlo, rhi;
+                const bool fast = bracket(sv, rlo, rhi);
                 cs[c] = sv;
+                cs[D + c] = fast ? rlo : 0.f;       // 0: no safe bracket, take the quotient
+                cs[2 * D + c] = fast ? rhi : 0.f;
                 if (it.blk == 0) reinterpret_cast<float *>(a.sv)[hc] = sv;
               }
             }
@@ -332,7 +346,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
     if (!go[i & 1]) break;
     mbar_try_wait(&full[s], par);                  // completed: orders this thread after the copy
     const QuantItem it = slot[s];
-    quant_tile<T, D, SCHEME>(a, it, reinterpret_cast<const T *>(smem + L::kTiles + s * L::kTileBytes), chan + s * D,
+    quant_tile<T, D, SCHEME>(a, it, reinterpret_cast<const T *>(smem + L::kTiles + s * L::kTileBytes),
+                             chan + s * kChanRows * D,
                              sc, &empty[s]);
   }
 }

@@ -55,6 +55,7 @@ struct QuantScratch {
   } red;
   float red_max[kQuantWarps];          // per-warp maxima of a quantisation block
   float row_scale[kBlockTokens];       // per-token Q scales of the tile (its rare exact path)
+  float2 e4m3_recip[256];              // NVFP4: bracket multipliers of 1/scale per E4M3 scale code
 };
 
 // 8 values (one 16-byte word) -> float, exact.
@@ -161,6 +162,18 @@ __device__ __forceinline__ void load_rows(const T *tile, int rows, int r0, int c
   for (int p = 0; p < kRowPasses<T, D>; ++p) {
     const int r = r0 + p * RPP;
     u[p] = r < rows ? *reinterpret_cast<const uint4 *>(tile + r * D + cg * 8) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The same rows, with row 0 (always valid) standing in for rows at and past
+// `rows`: a copy of valid data changes no maximum or minimum.
+template <typename T, int D>
+__device__ __forceinline__ void load_rows_dup(const T *tile, int rows, int r0, int cg, uint4 (&u)[kRowPasses<T, D>]) {
+  constexpr int RPP = kQuantConsumers / (D / 8);
+#pragma unroll
+  for (int p = 0; p < kRowPasses<T, D>; ++p) {
+    const int r = r0 + p * RPP;
+    u[p] = *reinterpret_cast<const uint4 *>(tile + (r < rows ? r : 0) * D + cg * 8);
   }
 }
 
@@ -330,40 +343,38 @@ __device__ __forceinline__ void qk_block_tile(const T *tile, int rows, const flo
 #pragma unroll
   for (int i = 0; i < 8; ++i) nmu[i] = IS_K ? -mu_s[cg * 8 + i] : 0.f;
   uint4 u[PASSES];
-  load_rows<T, D>(tile, rows, r0, cg, u);
+  load_rows_dup<T, D>(tile, rows, r0, cg, u);      // rows past `rows`: copies of row 0 (codes not stored)
 
+  const uint32_t w0[4] = {u[0].x, u[0].y, u[0].z, u[0].w};
   uint32_t hi[4], lo[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    hi[i] = IS_K ? Packed<T>::kNegInf : 0u;
-    lo[i] = Packed<T>::kPosInf;
+    hi[i] = IS_K ? w0[i] : 0u;
+    lo[i] = w0[i];
   }
 #pragma unroll
   for (int p = 0; p < PASSES; ++p) {
-    const bool valid = r0 + p * RPP < rows;        // a zero row is not data for the K extrema
     const uint32_t w[4] = {u[p].x, u[p].y, u[p].z, u[p].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       if (IS_K) {
-        hi[i] = max2<T>(hi[i], valid ? w[i] : Packed<T>::kNegInf);
-        lo[i] = min2<T>(lo[i], valid ? w[i] : Packed<T>::kPosInf);
+        hi[i] = max2<T>(hi[i], w[i]);
+        lo[i] = min2<T>(lo[i], w[i]);
       } else {
         hi[i] = absmax2<T>(hi[i], w[i]);
       }
     }
   }
   float amax = 0.f;
-  if (!IS_K || r0 < rows) {                        // no rows: no term (mu may be infinite)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 h = unpack2<T>(hi[i]);
-      if (IS_K) {
-        const float2 l = unpack2<T>(lo[i]);
-        amax = fmax3_nan(amax, __fadd_rn(h.x, nmu[2 * i]), __fsub_rn(-nmu[2 * i], l.x));
-        amax = fmax3_nan(amax, __fadd_rn(h.y, nmu[2 * i + 1]), __fsub_rn(-nmu[2 * i + 1], l.y));
-      } else {
-        amax = fmax3_nan(amax, h.x, h.y);
-      }
+  for (int i = 0; i < 4; ++i) {
+    const float2 h = unpack2<T>(hi[i]);
+    if (IS_K) {
+      const float2 l = unpack2<T>(lo[i]);
+      amax = fmax3_nan(amax, __fadd_rn(h.x, nmu[2 * i]), __fsub_rn(-nmu[2 * i], l.x));
+      amax = fmax3_nan(amax, __fadd_rn(h.y, nmu[2 * i + 1]), __fsub_rn(-nmu[2 * i + 1], l.y));
+    } else {
+      amax = fmax3_nan(amax, h.x, h.y);
     }
   }
 #pragma unroll
@@ -470,9 +481,12 @@ __device__ __forceinline__ bool bracket(float sv, float &rlo, float &rhi) {
   return r > 1.2e-38f && r < 1.0e38f;
 }
 
-// E4M3 codes of 4 values of one channel by the bracket; returns the codes of
-// the upper end and clears `ok` when the ends disagree.
-__device__ __forceinline__ uint32_t e4m3_codes4_fast(const float (&x)[4], float rlo, float rhi, bool &ok) {
+// E4M3 codes of 4 values of one channel by the bracket: returns the codes of
+// the upper end; sets bit j of `bad` where value j's two ends round apart
+// (the quotient then lies next to a rounding boundary, typically exactly on
+// it: bf16 values over a scale with few significant bits often land on an
+// E4M3 midpoint).
+__device__ __forceinline__ uint32_t e4m3_codes4_fast(const float (&x)[4], float rlo, float rhi, unsigned &bad) {
   const float2 a = make_float2(x[0], x[1]);
   const float2 b = make_float2(x[2], x[3]);
   const float2 alo = fmul2(a, make_float2(rlo, rlo));
@@ -481,7 +495,9 @@ __device__ __forceinline__ uint32_t e4m3_codes4_fast(const float (&x)[4], float 
   const float2 bhi = fmul2(b, make_float2(rhi, rhi));
   const uint32_t clo = cvt_e4m3x2(alo.x, alo.y) | (cvt_e4m3x2(blo.x, blo.y) << 16);
   const uint32_t chi = cvt_e4m3x2(ahi.x, ahi.y) | (cvt_e4m3x2(bhi.x, bhi.y) << 16);
-  ok = ok && clo == chi;
+  const uint32_t d = clo ^ chi;
+  bad = ((d & 0xFFu) != 0u) | (((d >> 8) & 0xFFu) != 0u) << 1 | (((d >> 16) & 0xFFu) != 0u) << 2 |
+        ((d >> 24) != 0u) << 3;
   return chi;
 }
 
@@ -493,7 +509,9 @@ __device__ __forceinline__ void store_codes(uint8_t *dst, const uint32_t (&w)[G]
     *reinterpret_cast<uint32_t *>(dst) = w[0];
 }
 
-// Per-channel FP8 E4M3 of a V tile (s_v = the stage's per-channel values),
+// Per-channel FP8 E4M3 of a V tile (the stage's per-channel values: s_v in
+// sv_s[0 .. d), the bracket multipliers of s_v in sv_s[d .. 2d) and [2d ..
+// 3d), 0 where 1/s_v has no safe bracket),
 // written transposed into vt_h[c * Nv + tok0 + t] for the tile's tokens below
 // Nv (tokens at and past N get code 0).  Warp w takes 4 TPT tokens of 64
 // channels; lane l the 8 channels 8 (l mod 8) .. + 7 of that half and the TPT
@@ -516,40 +534,30 @@ __device__ __forceinline__ void v_tile(const T *tile, int rows, int tok0, int Nv
 #pragma unroll
   for (int t = 0; t < TPT; ++t)
     raw[t] = t0 + t < rows ? *reinterpret_cast<const uint4 *>(tile + (t0 + t) * D + c0) : make_uint4(0u, 0u, 0u, 0u);
-  unsigned redo = 0u;
   if (tok0 + t0 < Nv) {                            // Nv is a multiple of 16: all TPT tokens in or out
+    uint64_t redo = 0u;                            // bit TPT i + t: channel c0 + i, token t0 + t
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float rlo, rhi;
-      bool ok = bracket(sv_s[c0 + i], rlo, rhi);
+      const float rlo = sv_s[D + c0 + i], rhi = sv_s[2 * D + c0 + i];
       uint32_t w[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float x[4] = {elem8<T>(raw[4 * g], i), elem8<T>(raw[4 * g + 1], i), elem8<T>(raw[4 * g + 2], i),
                             elem8<T>(raw[4 * g + 3], i)};
-        w[g] = e4m3_codes4_fast(x, rlo, rhi, ok);
+        unsigned bad;
+        w[g] = e4m3_codes4_fast(x, rlo, rhi, bad);
+        if (!(rlo > 0.f)) bad = 0xFu;              // no safe bracket for this channel
+        redo |= static_cast<uint64_t>(bad) << (TPT * i + 4 * g);
       }
-      if (!ok) redo |= 1u << i;
       store_codes<G>(vt_h + static_cast<size_t>(c0 + i) * Nv + tok0 + t0, w);
     }
-  }
-  // rare: channels with a code near a rounding boundary again, through the
-  // IEEE quotient (values from the stage)
-  for (; redo != 0u; redo &= redo - 1u) {
-    const int c = c0 + __ffs(redo) - 1;
-    const float sv = sv_s[c];
-    uint32_t w[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float q[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = t0 + 4 * g + j;
-        q[j] = t < rows ? __fdiv_rn(static_cast<float>(tile[t * D + c]), sv) : 0.f;
-      }
-      w[g] = cvt_e4m3x2(q[0], q[1]) | (cvt_e4m3x2(q[2], q[3]) << 16);
+    // values whose ends disagree: the code of the IEEE quotient, over the byte just stored
+    for (; redo != 0u; redo &= redo - 1u) {
+      const int e = __ffsll(static_cast<long long>(redo)) - 1;
+      const int c = c0 + e / TPT, t = t0 + e % TPT;
+      const float x = t < rows ? static_cast<float>(tile[t * D + c]) : 0.f;
+      vt_h[static_cast<size_t>(c) * Nv + tok0 + t] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x, sv_s[c]), 0.f));
     }
-    store_codes<G>(vt_h + static_cast<size_t>(c) * Nv + tok0 + t0, w);
   }
   release_stage(empty);
 }

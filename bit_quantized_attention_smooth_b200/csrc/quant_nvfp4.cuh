@@ -51,51 +51,67 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   return r;
 }
 
-// One NVFP4 block of 16 values: returns the E4M3 scale code and writes the 8
-// code bytes (as two 32-bit words), E2M1(x / scale) through the IEEE
-// quotient.  A block whose scale rounds to 0 (or is NaN) gets zero codes.
-__device__ __forceinline__ uint32_t nvfp4_block_exact(const float (&x)[16], uint32_t (&w)[2]) {
+// The bracket multipliers of 1/v for every E4M3 code v (entry = (RN(r (1 -
+// 2^-20)), RN(r (1 + 2^-20))), r = RN(1/v); (0, 0) for zero, NaN, negative
+// and codes without a safe bracket), one code per thread of the CTA's first
+// 256.
+__device__ __forceinline__ void fill_e4m3_recip(float2 *tab) {
+  if (threadIdx.x < 256) {
+    const float v = e4m3_to_float(threadIdx.x);
+    float rlo = 0.f, rhi = 0.f;
+    if (!(v > 0.f) || !bracket(v, rlo, rhi)) rlo = rhi = 0.f;
+    tab[threadIdx.x] = make_float2(rlo, rhi);
+  }
+}
+
+// One NVFP4 block of 16 values (reading: scale = E4M3_RNE(max|x| / 6), code =
+// E2M1_RNE_satfinite(x / scale), both quotients the IEEE float32 ones; a
+// scale of 0 or NaN gives zero codes), by brackets (see `bracket`): the
+// scale code from amax RN(RN(1/6) (1 -+ 2^-20)), both ends converted by one
+// instruction (when they differ, the quotient amax / 6 is computed); the
+// codes from x times the scale's entry of `recip`.  E4M3 and E2M1 rounding
+// are monotone, so equal codes at both ends are the quotient's codes.
+// Returns the scale code; w = the codes, two words of 8 nibbles (value k of
+// the block in nibble k mod 8 of word k / 8); bad[i] has bit 4 (k mod 8) set
+// where value k's two ends disagree (the caller then puts in the code of the
+// quotient, see nvfp4_code).
+__device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&x)[16], const float2 *recip, uint32_t (&w)[2],
+                                                     uint32_t (&bad)[2]) {
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmax_nan(amax, fabsf(x[i]));
-  const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
-  const float sc = e4m3_to_float(sc_code);
+  const uint32_t ends = cvt_e4m3x2(amax * __uint_as_float(0x3e2aaaa0u), amax * __uint_as_float(0x3e2aaab6u));
+  uint32_t sc_code = ends >> 8;
+  if ((ends & 0xFFu) != sc_code) sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
   w[0] = w[1] = 0u;
-  if (sc > 0.f) {
+  bad[0] = bad[1] = 0u;
+  if ((sc_code & 0x7Fu) == 0u || sc_code == 0x7Fu) return sc_code;   // zero scale, or NaN: zero codes
+  const float2 rr = recip[sc_code];
+  if (!(rr.x > 0.f)) {
+    bad[0] = bad[1] = 0x11111111u;
+    return sc_code;
+  }
+  uint32_t lo[2] = {0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const uint32_t b = cvt_e2m1x2(__fdiv_rn(x[i], sc), __fdiv_rn(x[i + 1], sc));
-      w[i >> 3] |= b << (4 * (i & 7));
-    }
+  for (int i = 0; i < 16; i += 2) {
+    const float2 pl = fmul2(make_float2(x[i], x[i + 1]), make_float2(rr.x, rr.x));
+    const float2 ph = fmul2(make_float2(x[i], x[i + 1]), make_float2(rr.y, rr.y));
+    lo[i >> 3] |= cvt_e2m1x2(pl.x, pl.y) << (4 * (i & 7));
+    w[i >> 3] |= cvt_e2m1x2(ph.x, ph.y) << (4 * (i & 7));
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    uint32_t d = lo[k] ^ w[k];
+    d |= d >> 1;
+    d |= d >> 2;
+    bad[k] = d & 0x11111111u;
   }
   return sc_code;
 }
 
-// The same block with the codes by the bracket of `bracket` (x RN(r (1 -+
-// 2^-20)), r = RN(1/scale)): E2M1 rounding is monotone, so equal codes at
-// both ends are the quotient's codes.  Clears `ok` when they differ (the
-// caller then takes nvfp4_block_exact).
-__device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&x)[16], uint32_t (&w)[2], bool &ok) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmax_nan(amax, fabsf(x[i]));
-  const uint32_t sc_code = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
-  const float sc = e4m3_to_float(sc_code);
-  w[0] = w[1] = 0u;
-  if (sc > 0.f) {
-    float rlo, rhi;
-    ok = bracket(sc, rlo, rhi) && ok;
-    uint32_t lo[2] = {0u, 0u};
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const float2 pl = fmul2(make_float2(x[i], x[i + 1]), make_float2(rlo, rlo));
-      const float2 ph = fmul2(make_float2(x[i], x[i + 1]), make_float2(rhi, rhi));
-      lo[i >> 3] |= cvt_e2m1x2(pl.x, pl.y) << (4 * (i & 7));
-      w[i >> 3] |= cvt_e2m1x2(ph.x, ph.y) << (4 * (i & 7));
-    }
-    ok = ok && lo[0] == w[0] && lo[1] == w[1];
-  }
-  return sc_code;
+// E2M1 code of x / scale through the IEEE quotient.
+__device__ __forceinline__ uint32_t nvfp4_code(float x, uint32_t sc_code) {
+  return cvt_e2m1x2(__fdiv_rn(x, e4m3_to_float(sc_code)), 0.f) & 0xFu;
 }
 
 // NVFP4 of a Q tile (IS_K = false) or of K - mu (IS_K = true, mu = the
@@ -104,8 +120,8 @@ __device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&x)[16], uint3
 // (row r at codes_blk + r d/2); the scale of every row (0 for rows past
 // `rows`) into the tile's scale-factor blocks sf_tile.
 template <typename T, int D, bool IS_K>
-__device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const float *mu_s, uint8_t *codes_blk,
-                                                uint8_t *sf_tile, uint64_t *empty) {
+__device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const float *mu_s, const float2 *recip,
+                                                uint8_t *codes_blk, uint8_t *sf_tile, uint64_t *empty) {
   constexpr int BPR = D / 16;                      // blocks per row
   constexpr int RPP = kQuantConsumers / BPR;
   constexpr int PASSES = kBlockTokens / RPP;
@@ -123,7 +139,6 @@ __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const f
     for (int h = 0; h < 2; ++h)
       u[p][h] = r < rows ? *reinterpret_cast<const uint4 *>(tile + r * D + b * 16 + 8 * h) : make_uint4(0u, 0u, 0u, 0u);
   }
-  unsigned redo = 0u;
 #pragma unroll
   for (int p = 0; p < PASSES; ++p) {
     const int r = r0 + p * RPP;
@@ -140,29 +155,20 @@ __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const f
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], mu[i]);
     }
-    uint32_t w[2];
-    bool ok = true;
-    const uint32_t sc_code = nvfp4_block_fast(v, w, ok);
-    if (!ok) redo |= 1u << p;
+    uint32_t w[2], bad[2];
+    const uint32_t sc_code = nvfp4_block_fast(v, recip, w, bad);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {                  // values next to an E2M1 rounding boundary
+      for (uint32_t m = bad[k]; m != 0u; m &= m - 1u) {
+        const int nib = (__ffs(m) - 1) >> 2;
+        const int j = 8 * k + nib;
+        float xj = static_cast<float>(tile[r * D + b * 16 + j]);
+        if (IS_K) xj = __fsub_rn(xj, mu_s[b * 16 + j]);
+        w[k] = (w[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
+      }
+    }
     if (r < rows) *reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8) = make_uint2(w[0], w[1]);
     sf_tile[(b >> 2) * 512 + sf_offset(r, b)] = static_cast<uint8_t>(sc_code);
-  }
-  // rare: blocks near a rounding boundary again, through the IEEE quotient (from the stage)
-  for (; redo != 0u; redo &= redo - 1u) {
-    const int r = r0 + (__ffs(redo) - 1) * RPP;
-    if (r >= rows) continue;
-    float v[16];
-    float a[8], c[8];
-    lds8<T>(tile + r * D + b * 16, a);
-    lds8<T>(tile + r * D + b * 16 + 8, c);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = IS_K ? __fsub_rn(a[i], mu[i]) : a[i];
-      v[8 + i] = IS_K ? __fsub_rn(c[i], mu[8 + i]) : c[i];
-    }
-    uint32_t w[2];
-    nvfp4_block_exact(v, w);
-    *reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8) = make_uint2(w[0], w[1]);
   }
   release_stage(empty);
 }
@@ -174,8 +180,8 @@ __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const f
 // (a warp reads 128 consecutive bytes of a row), and stores 16 code bytes
 // per channel.
 template <typename T, int D>
-__device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, int Nv, uint8_t *vt_h,
-                                             uint8_t *sf_tile, uint64_t *empty) {
+__device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, int Nv, const float2 *recip,
+                                             uint8_t *vt_h, uint8_t *sf_tile, uint64_t *empty) {
   constexpr int NCH = D / 64;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -191,7 +197,6 @@ __device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, 
       x[0][t] = f.x;
       x[1][t] = f.y;
     }
-    unsigned redo = 0u;
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
       uint32_t w[4];
@@ -200,10 +205,17 @@ __device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, 
         float blk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) blk[i] = x[ch][16 * h + i];
-        uint32_t wh[2];
-        bool ok = true;
-        const uint32_t sc_code = nvfp4_block_fast(blk, wh, ok);
-        if (!ok) redo |= 1u << (2 * ch + h);
+        uint32_t wh[2], bad[2];
+        const uint32_t sc_code = nvfp4_block_fast(blk, recip, wh, bad);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {              // values next to an E2M1 rounding boundary
+          for (uint32_t m = bad[k]; m != 0u; m &= m - 1u) {
+            const int nib = (__ffs(m) - 1) >> 2;
+            const int r = tg * 32 + 16 * h + 8 * k + nib;
+            const float xj = r < rows ? static_cast<float>(tile[r * D + c + ch]) : 0.f;
+            wh[k] = (wh[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
+          }
+        }
         w[2 * h] = wh[0];
         w[2 * h + 1] = wh[1];
         const int t16 = 2 * tg + h;                // 16-token block of the tile
@@ -212,22 +224,6 @@ __device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, 
       if (tok0 + tg * 32 < Nv)                     // Nv is a multiple of 32
         *reinterpret_cast<uint4 *>(vt_h + static_cast<size_t>(c + ch) * (Nv / 2) + (tok0 + tg * 32) / 2) =
             make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    // rare: blocks near a rounding boundary again, through the IEEE quotient (from the stage)
-    for (; redo != 0u; redo &= redo - 1u) {
-      const int k = __ffs(redo) - 1;
-      const int ch = k >> 1, h = k & 1;
-      float blk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = tg * 32 + 16 * h + i;
-        blk[i] = r < rows ? static_cast<float>(tile[r * D + c + ch]) : 0.f;
-      }
-      uint32_t wh[2];
-      nvfp4_block_exact(blk, wh);
-      if (tok0 + tg * 32 < Nv)
-        *reinterpret_cast<uint2 *>(vt_h + static_cast<size_t>(c + ch) * (Nv / 2) + (tok0 + tg * 32 + 16 * h) / 2) =
-            make_uint2(wh[0], wh[1]);
     }
   }
   release_stage(empty);

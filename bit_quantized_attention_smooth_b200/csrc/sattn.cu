@@ -201,6 +201,15 @@ int launch_quant(const void *q, const void *k, const void *v, int BH, int N, uin
   a.nv = L.nv;
   const long long items = quant_items(SCHEME, BH, L.nblk);
   const int grid = static_cast<int>(std::min<long long>(2LL * sms, items));
+  // Lag (in heads) between a head's statistics and its K/V codes: enough for
+  // the items in flight (about four per CTA) to fit in between, capped so that
+  // the K and V of the lagged heads (read once, re-read from L2) stay within
+  // 64 MB of the 126 MB L2.
+  const long long per_head = quant_stat_items(SCHEME, L.nblk) + L.nblk;   // |A(h)|
+  const long long kv_head = 2LL * N * D * static_cast<long long>(sizeof(T));
+  const long long want = (4LL * grid + per_head - 1) / per_head;
+  const long long cap = std::max<long long>(1, (64LL << 20) / kv_head);
+  a.lag = static_cast<int>(std::max<long long>(1, std::min(want, cap)));
   kern<<<grid, kQuantThreads, QuantSmem<D>::kAlloc, st>>>(a);
   g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
