@@ -5,7 +5,7 @@
 // per-channel V scale the column maximum of all of V before any V code, so K
 // and V are read twice: once for the statistics, once for the codes.  The
 // work is one queue of items, taken in ticket order by all CTAs; per head h:
-//   A(h) = statistics items of K (and, I8QK_F8PV, V) of h, then Q tiles of h
+//   A(h) = statistics items of K (then, I8QK_F8PV, of V) of h, then Q tiles of h
 //   B(h) = K tiles of h, then V tiles of h
 // A tile is 128 tokens x d of one tensor of one (b,h); a statistics item is
 // kStatBlocks consecutive tiles, reduced over the CTA and published once.
@@ -18,11 +18,12 @@
 // evict-last hint and every other read evict-first).  HBM then sees each
 // input byte once.
 //
-// A K or V tile waits for its head's statistics: at the end of every
+// A K (V) tile waits for its head's K (V) statistics: at the end of every
 // statistics item, each of the d/32 warps that add into the head's
-// accumulators fences its atomics and bumps done[h] once; before the K/V tile
-// is handed to the compute warps, the producer spins (bounded) until done[h]
-// reaches d/32 times the head's number of statistics items.  The queue order
+// accumulators fences its atomics and bumps the tensor's done counter of the
+// head once; before the K/V tile is handed to the compute warps, the producer
+// spins (bounded) until that counter reaches d/32 times the tensor's number
+// of statistics items.  The queue order
 // makes the wait finite: an item waits only for items with smaller tickets,
 // each already taken by a running CTA that processes its items in ticket
 // order (the tiles of one item in consecutive stages); the unfinished item
@@ -63,7 +64,7 @@ struct QuantArgs {
   float *mu;
   double *ksum;
   unsigned *vmax;
-  unsigned *done;              // [BH] statistics publications per head
+  unsigned *done;              // [2][BH] statistics publications per head: K, then V
   unsigned *ticket;            // next ticket
   int BH, N, nblk, nv;
   int lag;                     // heads whose statistics are read before B(0)
@@ -115,8 +116,9 @@ __host__ __device__ __forceinline__ QuantItem quant_item(int scheme, unsigned t,
   }
   if (in_a) {
     if (r < static_cast<unsigned>(nstat)) {
-      const int g = scheme == kSchemeNvfp4 ? static_cast<int>(r) : static_cast<int>(r >> 1);
-      it.kind = (scheme != kSchemeNvfp4 && (r & 1u)) ? kItemVStat : kItemKStat;
+      const int groups = (nblk + kStatBlocks - 1) / kStatBlocks;   // K statistics first, then V
+      const int g = static_cast<int>(r) % groups;
+      it.kind = static_cast<int>(r) < groups ? kItemKStat : kItemVStat;
       it.blk = g * kStatBlocks;
       it.nsub = nblk - it.blk < kStatBlocks ? nblk - it.blk : kStatBlocks;
     } else {
@@ -175,12 +177,12 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
     case kItemKStat:
       stat_tile<T, D, false>(tile, it.rows, it.sub == 0, sc, empty);
       if (it.sub == it.nsub - 1)
-        stat_publish<D, false>(sc, a.ksum + static_cast<size_t>(it.bh) * D, nullptr, a.done + it.bh);
+        stat_publish<D, false>(sc, a.ksum + static_cast<size_t>(it.bh) * D, nullptr, a.done + it.bh);   // K
       break;
     case kItemVStat:
       stat_tile<T, D, true>(tile, it.rows, it.sub == 0, sc, empty);
       if (it.sub == it.nsub - 1)
-        stat_publish<D, true>(sc, nullptr, a.vmax + static_cast<size_t>(it.bh) * D, a.done + it.bh);
+        stat_publish<D, true>(sc, nullptr, a.vmax + static_cast<size_t>(it.bh) * D, a.done + a.BH + it.bh);   // V
       break;
     case kItemQ:
       if (NV)
@@ -245,8 +247,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
     // barrier is arrived on: the compute warps find everything in shared
     // memory.
     const int lane = threadIdx.x & 31;
-    // every statistics item is published once per warp that issued accumulator atomics
-    const unsigned stats_target = static_cast<unsigned>(quant_stat_items(SCHEME, a.nblk)) * (D / 32);
+    // every statistics item of a tensor is published once per warp that issued accumulator atomics
+    const unsigned stats_target = static_cast<unsigned>((a.nblk + kStatBlocks - 1) / kStatBlocks) * (D / 32);
     uint64_t keep = 0, stream = 0;
     unsigned next = 0;
     if (lane == 0) {
@@ -292,7 +294,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
         }
         if (it.kind == kItemK || (!NV && it.kind == kItemV)) {
           bool ready = true;
-          if (lane == 0) ready = wait_count(a.done + it.bh, stats_target, abort_flag);
+          if (lane == 0)
+            ready = wait_count(a.done + (it.kind == kItemV ? a.BH : 0) + it.bh, stats_target, abort_flag);
           if (__shfl_sync(0xffffffffu, ready, 0)) {
             float *cs = chan + s * kChanRows * D;
 #pragma unroll

@@ -404,7 +404,7 @@ __device__ __forceinline__ void qk_block_tile(const T *tile, int rows, const flo
     uint2 codes;
     if (!int8_codes8_fast(f, rcp, codes)) redo |= 1u << p;
     const int r = r0 + p * RPP;
-    if (r < rows) *reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8) = codes;
+    if (r < rows) __stcs(reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8), codes);
   }
   // rare: rows near a rounding tie again, through the IEEE quotient (from the stage)
   for (; redo != 0u; redo &= redo - 1u) {
@@ -453,7 +453,7 @@ __device__ __forceinline__ void q_token_tile(const T *tile, int rows, QuantScrat
     if (cg == 0) sc.row_scale[r] = s;
     if (r < rows) {
       if (cg == 0) scale_blk[r] = s;
-      *reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8) = codes;
+      __stcs(reinterpret_cast<uint2 *>(out_blk + r * D + cg * 8), codes);
     }
   }
   __syncwarp();                                    // a row's lanes share a warp: its scale is visible
@@ -504,9 +504,9 @@ __device__ __forceinline__ uint32_t e4m3_codes4_fast(const float (&x)[4], float 
 template <int G>
 __device__ __forceinline__ void store_codes(uint8_t *dst, const uint32_t (&w)[G]) {
   if (G == 2)
-    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[G - 1]);
+    __stcs(reinterpret_cast<uint2 *>(dst), make_uint2(w[0], w[G - 1]));
   else
-    *reinterpret_cast<uint32_t *>(dst) = w[0];
+    __stcs(reinterpret_cast<unsigned int *>(dst), w[0]);
 }
 
 // Per-channel FP8 E4M3 of a V tile (the stage's per-channel values: s_v in

@@ -167,7 +167,7 @@ __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const f
         w[k] = (w[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
       }
     }
-    if (r < rows) *reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8) = make_uint2(w[0], w[1]);
+    if (r < rows) __stcs(reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8), make_uint2(w[0], w[1]));
     sf_tile[(b >> 2) * 512 + sf_offset(r, b)] = static_cast<uint8_t>(sc_code);
   }
   release_stage(empty);
@@ -222,8 +222,8 @@ __device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, 
         sf_tile[(t16 >> 2) * 512 + sf_offset(c + ch, t16)] = static_cast<uint8_t>(sc_code);
       }
       if (tok0 + tg * 32 < Nv)                     // Nv is a multiple of 32
-        *reinterpret_cast<uint4 *>(vt_h + static_cast<size_t>(c + ch) * (Nv / 2) + (tok0 + tg * 32) / 2) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        __stcs(reinterpret_cast<uint4 *>(vt_h + static_cast<size_t>(c + ch) * (Nv / 2) + (tok0 + tg * 32) / 2),
+               make_uint4(w[0], w[1], w[2], w[3]));
     }
   }
   release_stage(empty);

@@ -53,7 +53,8 @@ bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr
 bool is_nvfp4(int mode) { return base_mode(mode) == SATTN_NVFP4; }
 
 // The vmax section holds vmax[BH][d] and then the quantiser's work counters:
-// done[BH] and the ticket counter.  Offset of done from the section start.
+// done[2][BH] (K, V statistics) and the ticket counter.  Offset of done from
+// the section start.
 size_t counters_offset(size_t BH, int d) { return BH * d * sizeof(unsigned); }
 
 // NVFP4 workspace: q8/k8/vt8 hold the packed E2M1 codes of Q, K - mean and
@@ -73,7 +74,7 @@ sattn_ws_layout_t make_layout_nvfp4(int B, int H, int N, int d) {
   L.sv = off;   off = align_up(off + BH * L.nblk * 1024, kSectionAlign);
   L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.ksum = off; off += BH * d * sizeof(double);
-  L.vmax = off; off = align_up(off + counters_offset(BH, d) + (BH + 1) * sizeof(unsigned), kSectionAlign);
+  L.vmax = off; off = align_up(off + counters_offset(BH, d) + (2 * BH + 1) * sizeof(unsigned), kSectionAlign);
   L.total = off;
   return L;
 }
@@ -95,7 +96,7 @@ sattn_ws_layout_t make_layout_i8f8(int B, int H, int N, int d, bool per_token) {
   L.sv = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.mu = off;   off = align_up(off + BH * d * sizeof(float), kSectionAlign);
   L.ksum = off; off += BH * d * sizeof(double);
-  L.vmax = off; off = align_up(off + counters_offset(BH, d) + (BH + 1) * sizeof(unsigned), kSectionAlign);
+  L.vmax = off; off = align_up(off + counters_offset(BH, d) + (2 * BH + 1) * sizeof(unsigned), kSectionAlign);
   L.total = off;
   return L;
 }
@@ -194,7 +195,7 @@ int launch_quant(const void *q, const void *k, const void *v, int BH, int N, uin
   a.ksum = reinterpret_cast<double *>(ws + L.ksum);
   a.vmax = reinterpret_cast<unsigned *>(ws + L.vmax);
   a.done = reinterpret_cast<unsigned *>(ws + L.vmax + counters_offset(BH, D));
-  a.ticket = a.done + BH;
+  a.ticket = a.done + 2 * BH;
   a.BH = BH;
   a.N = N;
   a.nblk = L.nblk;

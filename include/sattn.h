@@ -240,7 +240,7 @@ int sattn_device_error(int clear);
  *              sq float32 [B*H, ceil(N/128)], or [B*H, N] with SATTN_Q_PER_TOKEN
  *              sk float32 [B*H, ceil(N/128)]   sv, mu float32 [B*H, d]
  *              ksum float64 [B*H, d], vmax uint32 [B*H, d] followed by
- *              the quantiser's work counters uint32 [B*H + 1] (scratch)
+ *              the quantiser's work counters uint32 [2*B*H + 1] (scratch)
  *   NVFP4 (same fields, other contents):
  *              q8, k8 E2M1 codes, two per byte (low nibble = even channel)
  *                        [B*H, N, d/2]
