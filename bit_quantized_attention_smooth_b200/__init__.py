@@ -30,7 +30,7 @@ STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
 # Every entry point declared in include/sattn.h.
 EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
            "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc",
-           "sattn_fwd_host", "sattn_kernel_launches", "sattn_debug_set_wait_limit",
+           "sattn_fwd_host", "sattn_kernel_launches", "sattn_debug_set_wait_limit", "sattn_debug_withhold_statistics",
            "sattn_fwd_quantized_sparse", "sattn_fwd_sparse")
 
 
@@ -79,6 +79,8 @@ def lib():
         L.sattn_kernel_launches.argtypes = [i]
         L.sattn_debug_set_wait_limit.restype = i
         L.sattn_debug_set_wait_limit.argtypes = [ctypes.c_longlong, i]
+        L.sattn_debug_withhold_statistics.restype = i
+        L.sattn_debug_withhold_statistics.argtypes = [i]
         L.sattn_fwd_quantized_sparse.restype = i
         L.sattn_fwd_quantized_sparse.argtypes = [vp, sz, vp, i, i, i, i, i, f, i, vp, vp]
         L.sattn_fwd_sparse.restype = i

@@ -57,6 +57,10 @@ struct QuantItem {
   int kind, bh, blk, rows, sub, nsub;
 };
 
+// Failure-path test hook: when non-zero, no head's statistics ever count as
+// ready (the producers' waits for them run out).
+__device__ int g_withhold_statistics = 0;
+
 struct QuantArgs {
   const void *q, *k, *v;
   uint8_t *q8, *k8, *vt8;      // codes
@@ -248,7 +252,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs
     // memory.
     const int lane = threadIdx.x & 31;
     // every statistics item of a tensor is published once per warp that issued accumulator atomics
-    const unsigned stats_target = static_cast<unsigned>((a.nblk + kStatBlocks - 1) / kStatBlocks) * (D / 32);
+    const unsigned stats_target = static_cast<unsigned>((a.nblk + kStatBlocks - 1) / kStatBlocks) * (D / 32) +
+                                  (g_withhold_statistics ? 1u : 0u);
     uint64_t keep = 0, stream = 0;
     unsigned next = 0;
     if (lane == 0) {

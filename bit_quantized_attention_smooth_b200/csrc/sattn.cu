@@ -621,6 +621,11 @@ int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile) {
   return SATTN_OK;
 }
 
+int sattn_debug_withhold_statistics(int on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(g_withhold_statistics, &v, sizeof(v)) == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+}
+
 unsigned long long sattn_kernel_launches(int reset) {
   return reset ? g_launches.exchange(0) : g_launches.load();
 }

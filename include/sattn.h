@@ -222,6 +222,15 @@ const char *sattn_status_string(int status);
  * device variables).  Returns SATTN_ERR_INVALID_ARG for withhold_k_tile < -1. */
 int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile);
 
+/* Failure-path test hook; not for production use.  With on != 0, the
+ * quantiser (sattn_quantize and every call that quantises) never sees a
+ * head's K/V statistics as complete: the waits for them run out after the
+ * bound set by sattn_debug_set_wait_limit, bit 0 of the device error word is
+ * set, the copies in flight complete and the kernel returns with the
+ * workspace partly written.  on == 0 restores normal operation.  Synchronous
+ * (it writes one device variable).  Returns SATTN_OK or SATTN_ERR_CUDA. */
+int sattn_debug_withhold_statistics(int on);
+
 /* Number of CUDA kernels this library has launched, in this process, since it
  * was loaded or since the last call with reset != 0 (which returns the count
  * and sets it to 0).  Counts launches (of every entry point, all devices), not

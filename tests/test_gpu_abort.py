@@ -1,4 +1,5 @@
-"""The bounded-wait failure path of the attention kernels, made to run on purpose.
+"""The bounded-wait failure paths of the attention kernels and the quantiser,
+made to run on purpose.
 
 Every wait between the roles of an attention kernel (copy producer, MMA issuer,
 softmax warps) gives up after a bound, records bit 0 of the device error word,
@@ -49,6 +50,41 @@ def test_wait_that_runs_out_sets_error_word_and_the_next_call_is_clean(mode, cau
     finally:
         assert L.sattn_debug_set_wait_limit(0, -1) == OK
     again = sattn.fwd(q, k, v, causal=causal, mode=mode)
+    torch.cuda.synchronize()
+    assert sattn.device_error() == 0
+    assert torch.equal(again, ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode", ["i8f8", "nvfp4"])
+def test_quantiser_statistics_wait_that_runs_out_sets_error_word_and_the_next_call_is_clean(mode):
+    """The quantiser's producers wait for a head's K/V statistics before they
+    hand out its K and V tiles.  The hook makes that count unreachable (a flag
+    that nothing sets); with a short bound every such wait runs out, the
+    kernel returns, and the next call with the hook off writes the same
+    workspace as before."""
+    assert torch.cuda.is_available(), "needs a CUDA device"
+    sattn_build.build()
+    L = sattn.lib()
+    w = W.custom(1, 2, 640, 128, seed=62)
+    q, k, v = W.make_inputs(w, "cuda")
+    lay = sattn.workspace_layout(w.B, w.H, w.N, w.d, mode=mode, dtype=q.dtype)
+    data = lay["ksum"]                               # codes and scales; the scratch after them differs
+    sattn.device_error(clear=True)
+    ref = sattn.quantize(q, k, v, mode=mode)[:data].clone()
+    torch.cuda.synchronize()
+    assert sattn.device_error() == 0
+    try:
+        assert L.sattn_debug_set_wait_limit(200_000, -1) == OK
+        assert L.sattn_debug_withhold_statistics(1) == OK
+        sattn.quantize(q, k, v, mode=mode)          # launches fine; the kernel gives up inside
+        torch.cuda.synchronize()                     # no fault: the kernel returned
+        word = sattn.device_error(clear=True)
+        assert word & 1, f"error word {word}: a statistics wait should have run out"
+    finally:
+        assert L.sattn_debug_withhold_statistics(0) == OK
+        assert L.sattn_debug_set_wait_limit(0, -1) == OK
+    again = sattn.quantize(q, k, v, mode=mode)[:data]
     torch.cuda.synchronize()
     assert sattn.device_error() == 0
     assert torch.equal(again, ref)
