@@ -435,6 +435,7 @@ def run_gpu(args):
                 tj = json.load(f)
             if tj.get("kernel_hash") == kernel_hash(mode) and tj.get("workload") == w.name:
                 traffic = tj.get("dram_bytes_per_launch_full")
+        quant = quantizer_roofline(sattn, w, q, mode, args.q_per_token, median(quant_ms), peaks, src)
         cpu = None
         if ws_n == 1 and not args.no_cpu_baseline:
             cpu_ops, cpu_s, rows_n = oracle_sample(w, args.cpu_seconds)
@@ -473,6 +474,7 @@ def run_gpu(args):
                          "peak_source": f"{src}: {PEAK_RATIO[mode]:.0f} x bf16 burst {peaks['bf16_tflops']} "
                                         f"(nominal dense ratio of {mode} to bf16)"},
             "roofline_mufu": mufu,
+            "roofline_quantize": quant,
             "cpu_baseline": cpu,
             "e2e": {"value": job_throughput(ops, ws_n, e2e_ms), "unit": "TOPS",
                     "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
@@ -489,13 +491,41 @@ def run_gpu(args):
     return 0
 
 
-def kernel_hash(mode="i8f8"):
+def kernel_hash(mode="i8f8", files=None):
+    """Hash of the sources a kernel is built from (the attention kernel of
+    `mode` by default): a recorded ncu traffic figure is reported only while
+    it matches."""
     import hashlib
     h = hashlib.sha256()
-    for f in (f"attn_{mode}.cuh", "ptx.cuh"):
+    for f in files or (f"attn_{mode}.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "bit_quantized_attention_smooth_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+QUANT_SOURCES = ("quant_fused.cuh", "quant_i8f8.cuh", "quant_nvfp4.cuh", "ptx.cuh")
+
+
+def quantizer_roofline(sattn, w, q, mode, q_per_token, quant_ms, peaks, src):
+    """HBM roofline of the quantiser (one launch, after one memset): its
+    algorithmic bytes are Q, K, V read once and the codes and scales written
+    once (the workspace sections before the scratch), over its device time."""
+    B, H, N, d = q.shape
+    lay = sattn.workspace_layout(B, H, N, d, mode=mode, dtype=q.dtype, q_per_token=q_per_token)
+    read = 3 * q.numel() * q.element_size()
+    write = lay["ksum"] - lay["q8"]
+    achieved = (read + write) / (quant_ms * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", f"quant_{mode}_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tj = json.load(f)
+        if (tj.get("kernel_hash") == kernel_hash(files=QUANT_SOURCES) and tj.get("workload") == w.name
+                and tj.get("q_per_token", False) == bool(q_per_token)):
+            traffic = tj.get("dram_bytes_per_launch_full")
+    return {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": read + write,
+            "ms": quant_ms, "peak_source": f"{src}: copy bandwidth"}
 
 
 def main():
