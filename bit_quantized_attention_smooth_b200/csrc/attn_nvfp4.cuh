@@ -421,25 +421,23 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         const float lsc = live ? __log2f(sc) : 0.f;
         const float2 nb2 = make_float2(-(moff + lsc), -(moff + lsc));
         float2 bsum = make_float2(0.f, 0.f);
-        uint32_t bytes[8];
+        float2 y[8];
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(sa[hb * 16 + i]), __uint_as_float(sa[hb * 16 + i + 1])),
-                                 cl2, nb2);
-          const float2 y = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          bsum = fadd2(bsum, y);
-          bytes[i >> 1] = cvt_e2m1x2(y.x, y.y);
+        for (int i = 0; i < 8; ++i) {
+          const float2 x = ffma2(
+              make_float2(__uint_as_float(sa[hb * 16 + 2 * i]), __uint_as_float(sa[hb * 16 + 2 * i + 1])), cl2, nb2);
+          y[i] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          bsum = fadd2(bsum, y[i]);
         }
+        w[2 * hb] = cvt_e2m1x8(y[0], y[1], y[2], y[3]);
+        w[2 * hb + 1] = cvt_e2m1x8(y[4], y[5], y[6], y[7]);
         if (live) psum = fmaf(sc, bsum.x + bsum.y, psum);
         else {
           // a block whose scale rounds to 0 has all-zero codes; its P2 values
           // (below 6 * 2^-10 of 2688) still count towards the row sum
-#pragma unroll
-          for (int i = 0; i < 8; ++i) bytes[i] = 0u;
+          w[2 * hb] = w[2 * hb + 1] = 0u;
           psum += (bsum.x + bsum.y);
         }
-        w[2 * hb] = __byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040), __byte_perm(bytes[2], bytes[3], 0x0040), 0x5410);
-        w[2 * hb + 1] = __byte_perm(__byte_perm(bytes[4], bytes[5], 0x0040), __byte_perm(bytes[6], bytes[7], 0x0040), 0x5410);
       }
       // 16 bytes = keys 32 kq .. 32 kq + 31; 64-byte swizzled K-major row
       *reinterpret_cast<uint4 *>(prow + ((kq ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -452,12 +450,23 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         uint32_t o[kQD];
         load_oin(o);
         const float2 a2 = make_float2(a_pend, a_pend), s2 = make_float2(s1_pend, s1_pend);
+        if (__all_sync(0xffffffffu, a_pend == 1.f)) {
+          // the usual case (no row's reference max moved): O_out += s1 O_in, one packed FMA per two columns
 #pragma unroll
-        for (int i = 0; i < kQD; i += 2) {
-          const float2 tt = fmul2(s2, make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])));
-          const float2 rr = ffma2(a2, make_float2(o_out[i], o_out[i + 1]), tt);
-          o_out[i] = rr.x;
-          o_out[i + 1] = rr.y;
+          for (int i = 0; i < kQD; i += 2) {
+            const float2 rr = ffma2(s2, make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                    make_float2(o_out[i], o_out[i + 1]));
+            o_out[i] = rr.x;
+            o_out[i + 1] = rr.y;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kQD; i += 2) {
+            const float2 tt = fmul2(s2, make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])));
+            const float2 rr = ffma2(a2, make_float2(o_out[i], o_out[i + 1]), tt);
+            o_out[i] = rr.x;
+            o_out[i + 1] = rr.y;
+          }
         }
       }
       l = fmaf(alpha, l, s1 * psum);

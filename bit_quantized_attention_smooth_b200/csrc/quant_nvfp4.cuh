@@ -51,6 +51,21 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   return r;
 }
 
+// Eight floats -> one word of eight E2M1 codes (RNE, saturating), the values
+// of a, b, c, d in that order from the lowest nibble up.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return r;
+}
+
 // The bracket multipliers of 1/v for every E4M3 code v (entry = (RN(r (1 -
 // 2^-20)), RN(r (1 + 2^-20))), r = RN(1/v); (0, 0) for zero, NaN, negative
 // and codes without a safe bracket), one code per thread of the CTA's first
@@ -91,13 +106,18 @@ __device__ __forceinline__ uint32_t nvfp4_block_fast(const float (&x)[16], const
     bad[0] = bad[1] = 0x11111111u;
     return sc_code;
   }
-  uint32_t lo[2] = {0u, 0u};
+  uint32_t lo[2];
 #pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    const float2 pl = fmul2(make_float2(x[i], x[i + 1]), make_float2(rr.x, rr.x));
-    const float2 ph = fmul2(make_float2(x[i], x[i + 1]), make_float2(rr.y, rr.y));
-    lo[i >> 3] |= cvt_e2m1x2(pl.x, pl.y) << (4 * (i & 7));
-    w[i >> 3] |= cvt_e2m1x2(ph.x, ph.y) << (4 * (i & 7));
+  for (int k = 0; k < 2; ++k) {
+    float2 pl[4], ph[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 v = make_float2(x[8 * k + 2 * j], x[8 * k + 2 * j + 1]);
+      pl[j] = fmul2(v, make_float2(rr.x, rr.x));
+      ph[j] = fmul2(v, make_float2(rr.y, rr.y));
+    }
+    lo[k] = cvt_e2m1x8(pl[0], pl[1], pl[2], pl[3]);
+    w[k] = cvt_e2m1x8(ph[0], ph[1], ph[2], ph[3]);
   }
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
