@@ -179,7 +179,7 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&s)[32], float c, float 
     const float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
     const float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
     sum2 = fadd2(sum2, fadd2(p01, p23));
-    w[q] = __byte_perm(cvt_e4m3x2(p01.x, p01.y), cvt_e4m3x2(p23.x, p23.y), 0x5410);
+    w[q] = cvt_e4m3x4(p01, p23);
   }
   *reinterpret_cast<uint4 *>(prow + ((c16 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   *reinterpret_cast<uint4 *>(prow + (((c16 + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);

@@ -328,6 +328,20 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Four floats -> one word of four E4M3 codes (round to nearest even,
+// saturate), a.x in the lowest byte: the two pair conversions land in the
+// halves of the word directly.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float2 a, float2 b) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 // Packed two-lane FP32 arithmetic (one instruction for two values).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;

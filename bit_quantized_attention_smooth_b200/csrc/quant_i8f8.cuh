@@ -493,8 +493,8 @@ __device__ __forceinline__ uint32_t e4m3_codes4_fast(const float (&x)[4], float 
   const float2 blo = fmul2(b, make_float2(rlo, rlo));
   const float2 ahi = fmul2(a, make_float2(rhi, rhi));
   const float2 bhi = fmul2(b, make_float2(rhi, rhi));
-  const uint32_t clo = cvt_e4m3x2(alo.x, alo.y) | (cvt_e4m3x2(blo.x, blo.y) << 16);
-  const uint32_t chi = cvt_e4m3x2(ahi.x, ahi.y) | (cvt_e4m3x2(bhi.x, bhi.y) << 16);
+  const uint32_t clo = cvt_e4m3x4(alo, blo);
+  const uint32_t chi = cvt_e4m3x4(ahi, bhi);
   const uint32_t d = clo ^ chi;
   bad = ((d & 0xFFu) != 0u) | (((d >> 8) & 0xFFu) != 0u) << 1 | (((d >> 16) & 0xFFu) != 0u) << 2 |
         ((d >> 24) != 0u) << 3;
