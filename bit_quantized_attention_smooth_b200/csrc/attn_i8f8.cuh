@@ -187,25 +187,30 @@ __device__ __forceinline__ void p_chunk(const uint32_t (&s)[32], float c, float 
 
 // One pass over an S tile: P~ codes of the row into its P line in shared
 // memory; returns the row's sum of c_P P~ and (into xmax2) its largest
-// exponent argument x = S2 - m + log2 c_P.
+// exponent argument x = S2 - m + log2 c_P.  S is read W columns per TMEM
+// round trip (W = 64: fewer waits, more live registers; the causal kernels
+// run faster with W = 32, the others with W = 64, measured).
+template <int W>
 __device__ __forceinline__ float p_pass(uint32_t s_tmem, float c, float b, uint8_t *prow, int r, bool masked, int kv0,
                                         int N, bool causal, int row_g, float2 &xmax2) {
+  static_assert(W == 32 || W == 64, "columns per TMEM round trip");
+  constexpr int G = W / 32;                       // 32-column loads per wait
   float2 tsum2 = make_float2(0.f, 0.f);
 #pragma unroll 1
-  for (int hh = 0; hh < 2; ++hh) {
-    uint32_t s0[32], s1[32];
-    tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
-    tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
-    tmem_ld_wait(s0);
-    tmem_ld_wait(s1);
-    if (masked) {
-      mask_chunk(s0, kv0 + hh * 64, N, causal, row_g);
-      mask_chunk(s1, kv0 + hh * 64 + 32, N, causal, row_g);
-      p_chunk<true, true>(s0, c, b, prow, hh * 4, r, tsum2, xmax2);
-      p_chunk<true, true>(s1, c, b, prow, hh * 4 + 2, r, tsum2, xmax2);
-    } else {
-      p_chunk<false, true>(s0, c, b, prow, hh * 4, r, tsum2, xmax2);
-      p_chunk<false, true>(s1, c, b, prow, hh * 4 + 2, r, tsum2, xmax2);
+  for (int hh = 0; hh < kTile / W; ++hh) {
+    uint32_t sc[G][32];
+#pragma unroll
+    for (int g = 0; g < G; ++g) tmem_ld_32x32b_x32(s_tmem + hh * W + g * 32, sc[g]);
+#pragma unroll
+    for (int g = 0; g < G; ++g) tmem_ld_wait(sc[g]);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (masked) {
+        mask_chunk(sc[g], kv0 + hh * W + g * 32, N, causal, row_g);
+        p_chunk<true, true>(sc[g], c, b, prow, (hh * W + g * 32) / 16, r, tsum2, xmax2);
+      } else {
+        p_chunk<false, true>(sc[g], c, b, prow, (hh * W + g * 32) / 16, r, tsum2, xmax2);
+      }
     }
   }
   return tsum2.x + tsum2.y;
@@ -464,7 +469,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // which only serves to find the tile's row max)
       const float m_try = n > 0 ? m_ref : 0.f;
       float2 xm2 = make_float2(-INFINITY, -INFINITY);
-      float tsum = p_pass(s_tmem, c, m_try - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
+      float tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_try - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
       // x = S2 - m + log2 c_P;  the row max moves when S2max - m > tau  <=>  xmax > log2 448
       const float xmax = fmaxf(xm2.x, xm2.y);
       const bool up = n == 0 || xmax > kLog2_448;
@@ -473,7 +478,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (moved) {
         if (up) m_new = fmaxf(m_ref, xmax + (m_try - kLog2_CP));   // the tile's row max
         alpha = n > 0 ? ex2_approx(m_ref - m_new) : 0.f;
-        tsum = p_pass(s_tmem, c, m_new - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
+        tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_new - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
       }
       tc_fence_before();
       __syncwarp();
