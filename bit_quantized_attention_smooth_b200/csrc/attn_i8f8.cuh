@@ -194,22 +194,36 @@ template <int W>
 __device__ __forceinline__ float p_pass(uint32_t s_tmem, float c, float b, uint8_t *prow, int r, bool masked, int kv0,
                                         int N, bool causal, int row_g, float2 &xmax2) {
   static_assert(W == 32 || W == 64, "columns per TMEM round trip");
-  constexpr int G = W / 32;                       // 32-column loads per wait
   float2 tsum2 = make_float2(0.f, 0.f);
+  if constexpr (W == 64) {
 #pragma unroll 1
-  for (int hh = 0; hh < kTile / W; ++hh) {
-    uint32_t sc[G][32];
-#pragma unroll
-    for (int g = 0; g < G; ++g) tmem_ld_32x32b_x32(s_tmem + hh * W + g * 32, sc[g]);
-#pragma unroll
-    for (int g = 0; g < G; ++g) tmem_ld_wait(sc[g]);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int hh = 0; hh < 2; ++hh) {
+      uint32_t s0[32], s1[32];
+      tmem_ld_32x32b_x32(s_tmem + hh * 64, s0);
+      tmem_ld_32x32b_x32(s_tmem + hh * 64 + 32, s1);
+      tmem_ld_wait(s0);
+      tmem_ld_wait(s1);
       if (masked) {
-        mask_chunk(sc[g], kv0 + hh * W + g * 32, N, causal, row_g);
-        p_chunk<true, true>(sc[g], c, b, prow, (hh * W + g * 32) / 16, r, tsum2, xmax2);
+        mask_chunk(s0, kv0 + hh * 64, N, causal, row_g);
+        mask_chunk(s1, kv0 + hh * 64 + 32, N, causal, row_g);
+        p_chunk<true, true>(s0, c, b, prow, hh * 4, r, tsum2, xmax2);
+        p_chunk<true, true>(s1, c, b, prow, hh * 4 + 2, r, tsum2, xmax2);
       } else {
-        p_chunk<false, true>(sc[g], c, b, prow, (hh * W + g * 32) / 16, r, tsum2, xmax2);
+        p_chunk<false, true>(s0, c, b, prow, hh * 4, r, tsum2, xmax2);
+        p_chunk<false, true>(s1, c, b, prow, hh * 4 + 2, r, tsum2, xmax2);
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int hh = 0; hh < 4; ++hh) {
+      uint32_t s0[32];
+      tmem_ld_32x32b_x32(s_tmem + hh * 32, s0);
+      tmem_ld_wait(s0);
+      if (masked) {
+        mask_chunk(s0, kv0 + hh * 32, N, causal, row_g);
+        p_chunk<true, true>(s0, c, b, prow, hh * 2, r, tsum2, xmax2);
+      } else {
+        p_chunk<false, true>(s0, c, b, prow, hh * 2, r, tsum2, xmax2);
       }
     }
   }
