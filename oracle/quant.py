@@ -165,3 +165,18 @@ def quantize_head_nvfp4(q32, k32, v32):
     return dict(mu=mu, q=qc, q_sc=qsc, q_sc_codes=qsc_codes,
                 k=kc, k_sc=ksc, k_sc_codes=ksc_codes,
                 vt=vc, vt_sc=vsc, vt_sc_codes=vsc_codes)
+
+
+def quantize_head_mxfp4(q32, k32, v32):
+    """All quantised operands of one head for the MXFP4 ablation of the NVFP4
+    mode (tag page, SageAttention3 summary, FP4 bullet [15]): the operands of
+    ``quantize_head_nvfp4`` with blocks of 32 values and E8M0 scale codes
+    (``mxfp4_quant_rows``); V blocked along tokens and returned transposed."""
+    mu = k_channel_mean(k32)
+    kp = smooth_k(k32, mu)
+    qc, qsc_codes, qsc = mxfp4_quant_rows(q32)
+    kc, ksc_codes, ksc = mxfp4_quant_rows(kp)
+    vc, vsc_codes, vsc = mxfp4_quant_rows(np.ascontiguousarray(v32.T))
+    return dict(mu=mu, q=qc, q_sc=qsc, q_sc_codes=qsc_codes,
+                k=kc, k_sc=ksc, k_sc_codes=ksc_codes,
+                vt=vc, vt_sc=vsc, vt_sc_codes=vsc_codes)

@@ -72,3 +72,24 @@ def test_nvfp4_is_more_accurate_than_mxfp4(w, rows):
     c_nv, c_mx = A.cosine(e, nv), A.cosine(e, mx)
     print(f"{w.name}: cos NVFP4 {c_nv:.5f}  MXFP4 {c_mx:.5f}")
     assert c_nv > c_mx
+
+
+def test_quantize_head_mxfp4_matches_the_emulations_operands():
+    """The per-head MXFP4 operands (the quantiser's target on the GPU) decode to
+    the operands the MXFP4 emulation multiplies: Q, K - mean along channels, V
+    along tokens; every block's largest magnitude lies in [4, 8) x its scale."""
+    w = W.custom(1, 1, 77, 64, seed=82)
+    q, k, v = (t[0, 0].float().numpy() for t in W.make_inputs(w))
+    z = Qz.quantize_head_mxfp4(q, k, v)
+    kp = Qz.smooth_k(k, Qz.k_channel_mean(k))
+    for key, x in (("q", q), ("k", kp), ("vt", np.ascontiguousarray(v.T))):
+        deq = Qz.nvfp4_dequant_rows(z[key], z[key + "_sc"], block=32)
+        assert np.array_equal(deq[:, :x.shape[1]], Qz.fp4_rows(x, "mxfp4")[:, :x.shape[1]])
+        xp = np.zeros(deq.shape)
+        xp[:, :x.shape[1]] = x
+        amax = np.abs(xp.reshape(xp.shape[0], -1, 32)).max(axis=2)
+        sc = e8m0_decode(z[key + "_sc_codes"])
+        live = amax > 0
+        assert np.all((4 * sc[live] <= amax[live]) & (amax[live] < 8 * sc[live]))
+    # V padded with zero tokens up to a multiple of 32
+    assert z["vt"].shape == (64, 96) and not np.any(e2m1_decode(z["vt"][:, 77:]))
