@@ -8,7 +8,7 @@ starts; L2 is flushed (a 256 MiB write) between steps, outside the per-step
 events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--mode i8f8|nvfp4] [--workload NAME] [--causal] [--q-per-token]
+                    [--mode i8f8|nvfp4|mxfp4] [--workload NAME] [--causal] [--q-per-token]
     python bench.py --sweep [--steps K]      # the B=4 H=32 sweep, both modes
 
 Prints ONE JSON line on rank 0 (the sweep: one per point and mode).  Step and
@@ -203,8 +203,8 @@ def run_reference(args):
 
 # ---------------------------------------------------------------------------- GPU arm
 
-PEAK_RATIO = {"i8f8": 2.0, "nvfp4": 4.0}       # dense INT8/FP8 = 2 x bf16, FP4 = 4 x bf16 (nominal)
-DATASHEET = {"i8f8": 4500.0, "nvfp4": 9000.0}  # dense TOPS
+PEAK_RATIO = {"i8f8": 2.0, "nvfp4": 4.0, "mxfp4": 4.0}   # dense INT8/FP8 = 2 x bf16, FP4 = 4 x bf16 (nominal)
+DATASHEET = {"i8f8": 4500.0, "nvfp4": 9000.0, "mxfp4": 9000.0}  # dense TOPS
 
 
 def median(xs):
@@ -385,7 +385,7 @@ def run_gpu(args):
     # the other mode on the same inputs, and per-token Q scales (I8QK_F8PV), beside the headline
     legs = {}
     for name, (m, qtok) in {"nvfp4": ("nvfp4", False), "i8f8": ("i8f8", False),
-                            "i8f8_q_per_token": ("i8f8", True)}.items():
+                            "i8f8_q_per_token": ("i8f8", True), "mxfp4": ("mxfp4", False)}.items():
         if m == mode and qtok == args.q_per_token:
             continue
         r = ModeRunner(sattn, q, k, v, causal, m, qtok, flush)
@@ -426,7 +426,7 @@ def run_gpu(args):
         att = attention_report(w, mode, causal, attn_med, peaks)
         achieved = att["tops"]
         for name, leg in legs.items():
-            m = "nvfp4" if name == "nvfp4" else "i8f8"
+            m = name if name in ("nvfp4", "mxfp4") else "i8f8"
             leg["attention_kernel"] = attention_report(w, m, causal, leg.pop("attention_kernel_ms"), peaks)
         traffic = None
         tpath = os.path.join(ROOT, "profiles", f"attn_{mode}_traffic.json")
@@ -454,10 +454,11 @@ def run_gpu(args):
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("int8 QK^T / e4m3 PV (fp32 softmax + accumulation)" if mode == "i8f8"
-                      else "nvfp4 QK^T / nvfp4 PV (e2m1 + e4m3 block scales; fp32 softmax + accumulation)"),
+            "dtype": {"i8f8": "int8 QK^T / e4m3 PV (fp32 softmax + accumulation)",
+                      "nvfp4": "nvfp4 QK^T / nvfp4 PV (e2m1 + e4m3 block scales; fp32 softmax + accumulation)",
+                      "mxfp4": "mxfp4 QK^T / mxfp4 PV (e2m1 + e8m0 block scales; fp32 softmax + accumulation)"}[mode],
             "data": "synthetic",
-            "config": {"workload": w.name, "mode": "I8QK_F8PV" if mode == "i8f8" else "NVFP4", "B": w.B, "H": w.H,
+            "config": {"workload": w.name, "mode": {"i8f8": "I8QK_F8PV", "nvfp4": "NVFP4", "mxfp4": "MXFP4"}[mode], "B": w.B, "H": w.H,
                        "N": w.N, "d": w.d, "causal": causal, "io_dtype": w.dtype,
                        "q_scales": "per token" if args.q_per_token else "per 128-token block",
                        "lazy_max_tau": sattn.I8F8_LAZY_TAU if mode == "i8f8" else None,
@@ -497,7 +498,7 @@ def kernel_hash(mode="i8f8", files=None):
     it matches."""
     import hashlib
     h = hashlib.sha256()
-    for f in files or (f"attn_{mode}.cuh", "ptx.cuh"):
+    for f in files or (f"attn_{'i8f8' if mode == 'i8f8' else 'nvfp4'}.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "bit_quantized_attention_smooth_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -536,7 +537,7 @@ def main():
     ap.add_argument("--impl", default="sattn", choices=["sattn", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="i8f8", choices=["i8f8", "nvfp4"])
+    ap.add_argument("--mode", default="i8f8", choices=["i8f8", "nvfp4", "mxfp4"])
     ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(W.WORKLOADS))
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--q-per-token", action="store_true", help="I8QK_F8PV with one Q scale per token")

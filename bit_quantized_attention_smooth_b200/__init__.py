@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsattn.so")
 
-MODES = {"i8f8": 0, "nvfp4": 1}
+MODES = {"i8f8": 0, "nvfp4": 1, "mxfp4": 2}
 FP16_IO = 0x100
 Q_PER_TOKEN = 0x200
 # Lazy reference-max threshold of the I8QK_F8PV kernel (SATTN_I8F8_LAZY_TAU in

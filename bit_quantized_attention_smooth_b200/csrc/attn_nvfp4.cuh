@@ -107,7 +107,8 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T with NVFP4 operands and UE4M3 block scales in TMEM.
+// D[tmem] (+)= A[smem] * B[smem]^T with E2M1 operands and one block scale per
+// 16 values in TMEM (UE4M3, or UE8M0 when the descriptor's bit 23 is set).
 __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
@@ -120,7 +121,7 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint
 }
 
 // Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format 1) K-major,
-// UE4M3 scales (bit 23 = 0), N >> 3 in [17,23), M >> 4 in [24,29), scale ids 0,
+// UE4M3 scales (bit 23 = 0; the MXFP4 variant sets it for UE8M0), N >> 3 in [17,23), M >> 4 in [24,29), scale ids 0,
 // dense K = 64.
 __host__ __device__ constexpr uint32_t idesc_nvfp4(int M, int N) {
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
@@ -136,7 +137,12 @@ __device__ __forceinline__ uint64_t sdesc_f4(uint32_t smem_addr) {
          (uint64_t(1) << 46) | (mode << 61);
 }
 
-template <int D, bool CAUSAL, typename OutT, bool SPARSE>
+// MX = true: the MXFP4 ablation (tag page, SageAttention3 summary, FP4 bullet
+// [15]): every FP4 operand in blocks of 32 with E8M0 scales.  The MMA runs in
+// its 16-value scale mode with UE8M0 scales (each 32-block's scale stored
+// twice), which computes the same products; P's second stage takes the E8M0
+// scale of its 32-key block.
+template <int D, bool CAUSAL, typename OutT, bool SPARSE, bool MX = false>
 __global__ void __launch_bounds__(kF4Threads, 1)
     attn_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const AttnF4Args args) {
@@ -266,8 +272,9 @@ __global__ void __launch_bounds__(kF4Threads, 1)
   } else if (warp == 17) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdQK = idesc_nvfp4(kTile, kTile);
-      constexpr uint32_t kIdPV = idesc_nvfp4(kTile, D);
+      constexpr uint32_t kScaleE8M0 = MX ? (1u << 23) : 0u;   // scale format bit: UE8M0
+      constexpr uint32_t kIdQK = idesc_nvfp4(kTile, kTile) | kScaleE8M0;
+      constexpr uint32_t kIdPV = idesc_nvfp4(kTile, D) | kScaleE8M0;
       const uint32_t sQ = smem_u32(smem + L::kQ);
       bool ok = mbar_wait(q_full, 0, abort_flag);
       if (ok) {
@@ -407,6 +414,34 @@ __global__ void __launch_bounds__(kF4Threads, 1)
       float psum = 0.f;
       const float2 cl2 = make_float2(cl, cl);
       uint32_t w[4];
+      if constexpr (MX) {
+        // MXFP4: the quarter's 32 keys are one block; scale = 2^(floor(log2 max P2) - 2),
+        // its E8M0 code the biased exponent of max P2 minus 2 (0 below 2^-124),
+        // stored in both 16-key slots the MMA reads.  P2 / scale = 2^(S2 - moff
+        // - log2 scale) with an integer log2 scale.
+        const float p2max = ex2_approx(fmaf(fmaxf(bmax[0], bmax[1]), cl, -moff));
+        const uint32_t e = (__float_as_uint(p2max) >> 23) & 0xFFu;
+        const uint32_t sc_code = e > 2u ? e - 2u : 0u;
+        *reinterpret_cast<uint16_t *>(psf + sf_offset(r, (kq & 1) * 2)) = static_cast<uint16_t>(sc_code * 0x101u);
+        const float lsc = static_cast<float>(static_cast<int>(sc_code) - 127);
+        const float sc = sc_code != 0u ? __uint_as_float(sc_code << 23) : __uint_as_float(1u << 22);
+        const float2 nb2 = make_float2(-(moff + lsc), -(moff + lsc));
+        float2 bsum = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          float2 y[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float2 x = ffma2(
+                make_float2(__uint_as_float(sa[hb * 16 + 2 * i]), __uint_as_float(sa[hb * 16 + 2 * i + 1])), cl2, nb2);
+            y[i] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            bsum = fadd2(bsum, y[i]);
+          }
+          w[2 * hb] = cvt_e2m1x8(y[0], y[1], y[2], y[3]);
+          w[2 * hb + 1] = cvt_e2m1x8(y[4], y[5], y[6], y[7]);
+        }
+        psum = sc * (bsum.x + bsum.y);
+      } else {
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         const int blk = (kq & 1) * 2 + hb;                // 16-key block within the 64-key slice
@@ -438,6 +473,7 @@ __global__ void __launch_bounds__(kF4Threads, 1)
           w[2 * hb] = w[2 * hb + 1] = 0u;
           psum += (bsum.x + bsum.y);
         }
+      }
       }
       // 16 bytes = keys 32 kq .. 32 kq + 31; 64-byte swizzled K-major row
       *reinterpret_cast<uint4 *>(prow + ((kq ^ ((r >> 1) & 3)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);

@@ -47,7 +47,13 @@ constexpr int kQuantThreads = kQuantConsumers + 32;
 constexpr int kStatBlocks = 8;         // 128-token blocks per statistics item
 constexpr int kChanRows = 3;           // per-channel values a stage carries
 
-enum QuantScheme : int { kSchemeI8Block = 0, kSchemeI8Token = 1, kSchemeNvfp4 = 2 };
+enum QuantScheme : int { kSchemeI8Block = 0, kSchemeI8Token = 1, kSchemeNvfp4 = 2, kSchemeMxfp4 = 3 };
+
+// The FP4 schemes (NVFP4 and its MXFP4 ablation) share the tiles, the layout
+// and the queue: K statistics only (V needs no per-channel scale).
+__host__ __device__ constexpr bool fp4_scheme(int scheme) {
+  return scheme == kSchemeNvfp4 || scheme == kSchemeMxfp4;
+}
 enum QuantItemKind : int { kItemKStat = 0, kItemVStat = 1, kItemQ = 2, kItemK = 3, kItemV = 4, kItemEnd = 5 };
 
 // A queue item, or (in a stage slot) one tile of it: blocks blk .. blk +
@@ -77,7 +83,7 @@ struct QuantArgs {
 // Statistics items per head: K (and, I8QK_F8PV, V) in groups of kStatBlocks blocks.
 __host__ __device__ __forceinline__ int quant_stat_items(int scheme, int nblk) {
   const int groups = (nblk + kStatBlocks - 1) / kStatBlocks;
-  return scheme == kSchemeNvfp4 ? groups : 2 * groups;
+  return fp4_scheme(scheme) ? groups : 2 * groups;
 }
 
 // Number of items in the queue.
@@ -173,7 +179,8 @@ __device__ __forceinline__ bool wait_count(const unsigned *count, unsigned targe
 template <typename T, int D, int SCHEME>
 __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &it, const T *tile, const float *cs,
                                            QuantScratch<D> &sc, uint64_t *empty) {
-  constexpr bool NV = SCHEME == kSchemeNvfp4;
+  constexpr bool NV = fp4_scheme(SCHEME);
+  constexpr bool MX = SCHEME == kSchemeMxfp4;
   const size_t hrow = static_cast<size_t>(it.bh) * a.N;   // first row of the head
   const int tok0 = it.blk * kBlockTokens;
   const size_t sblk = static_cast<size_t>(it.bh) * a.nblk + it.blk;
@@ -190,7 +197,7 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
       break;
     case kItemQ:
       if (NV)
-        nvfp4_rows_tile<T, D, false>(tile, it.rows, cs, sc.e4m3_recip, a.q8 + (hrow + tok0) * (D / 2),
+        nvfp4_rows_tile<T, D, false, MX>(tile, it.rows, cs, sc.e4m3_recip, a.q8 + (hrow + tok0) * (D / 2),
                                      a.sq + sblk * (D / 64) * 512, empty);
       else if (SCHEME == kSchemeI8Token)
         q_token_tile<T, D>(tile, it.rows, sc, reinterpret_cast<int8_t *>(a.q8) + (hrow + tok0) * D,
@@ -201,7 +208,7 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
       break;
     case kItemK:
       if (NV)
-        nvfp4_rows_tile<T, D, true>(tile, it.rows, cs, sc.e4m3_recip, a.k8 + (hrow + tok0) * (D / 2),
+        nvfp4_rows_tile<T, D, true, MX>(tile, it.rows, cs, sc.e4m3_recip, a.k8 + (hrow + tok0) * (D / 2),
                                     a.sk + sblk * (D / 64) * 512, empty);
       else
         qk_block_tile<T, D, true>(tile, it.rows, cs, sc, reinterpret_cast<int8_t *>(a.k8) + (hrow + tok0) * D,
@@ -209,7 +216,7 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
       break;
     default:   // kItemV
       if (NV)
-        nvfp4_v_tile<T, D>(tile, it.rows, tok0, a.nv, sc.e4m3_recip,
+        nvfp4_v_tile<T, D, MX>(tile, it.rows, tok0, a.nv, sc.e4m3_recip,
                            a.vt8 + static_cast<size_t>(it.bh) * D * (a.nv / 2), a.sv + sblk * 1024, empty);
       else
         v_tile<T, D>(tile, it.rows, tok0, a.nv, cs, a.vt8 + static_cast<size_t>(it.bh) * D * a.nv, empty);
@@ -220,7 +227,7 @@ __device__ __forceinline__ void quant_tile(const QuantArgs &a, const QuantItem &
 template <typename T, int D, int SCHEME>
 __global__ void __launch_bounds__(kQuantThreads, 2) quant_kernel(const QuantArgs a) {
   using L = QuantSmem<D>;
-  constexpr bool NV = SCHEME == kSchemeNvfp4;
+  constexpr bool NV = fp4_scheme(SCHEME);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   QuantScratch<D> &sc = *reinterpret_cast<QuantScratch<D> *>(smem + L::kScratch);

@@ -12,6 +12,15 @@
 //           scale rounds to 0 gets zero codes.
 // Codes are packed two per byte, the lower-index value in the low nibble.
 //
+// The MXFP4 mode (the format the same bullet [15] compares NVFP4 with; OCP
+// Microscaling) uses the same tiles with blocks of 32 values (32 channels of a
+// Q/K token, 32 tokens of a V channel) and one E8M0 scale per block:
+//   scale = 2^(floor(log2 max|x|) - 2)  (E8M0 code = biased exponent of max|x| - 2,
+//           0 for max|x| < 2^-124, 255 = NaN);
+//   code  = E2M1_RNE_satfinite(x * 2^(127 - scale code))  (exact: a power of two).
+// The MMA reads the E8M0 scale per 16 values, so each block's code is stored
+// in both of its 16-value slots of the layout below.
+//
 // Scale factors are written directly in the layout the block-scaled MMA reads
 // after a 32x128b.warpx4 tensor-memory copy: for every 128-row tile and every
 // 64-value slice kk of the contraction axis, a 512-byte block in which the
@@ -134,12 +143,47 @@ __device__ __forceinline__ uint32_t nvfp4_code(float x, uint32_t sc_code) {
   return cvt_e2m1x2(__fdiv_rn(x, e4m3_to_float(sc_code)), 0.f) & 0xFu;
 }
 
+// E8M0 code of the MXFP4 scale of a block with largest magnitude amax (>= 0
+// or NaN): floor(log2 amax) - 2 + 127 = (biased exponent of amax) - 2, at
+// least 0 (amax below 2^-124, zero included; the codes are then 0 or exact
+// small values); NaN -> 255.  A finite float32 amax gives at most 253.
+__device__ __forceinline__ uint32_t mx_scale_code(float amax) {
+  if (amax != amax) return 255u;
+  const uint32_t e = (__float_as_uint(amax) >> 23) & 0xFFu;
+  return e > 2u ? e - 2u : 0u;
+}
+
+// 2^(127 - code) for a scale code in [0, 253]: the exact reciprocal of the scale.
+__device__ __forceinline__ float mx_inv_scale(uint32_t code) { return __uint_as_float((254u - code) << 23); }
+
+// E2M1 codes of 16 values of an MXFP4 block with scale code `code`: x times
+// the exact reciprocal, RNE satfinite; two words of 8 nibbles as in
+// nvfp4_block_fast.  A NaN scale gives zero codes.
+__device__ __forceinline__ void mxfp4_codes16(const float (&x)[16], uint32_t code, uint32_t (&w)[2]) {
+  if (code == 255u) {
+    w[0] = w[1] = 0u;
+    return;
+  }
+  const float r = mx_inv_scale(code);
+  const float2 r2 = make_float2(r, r);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    float2 p[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) p[j] = fmul2(make_float2(x[8 * k + 2 * j], x[8 * k + 2 * j + 1]), r2);
+    w[k] = cvt_e2m1x8(p[0], p[1], p[2], p[3]);
+  }
+}
+
 // NVFP4 of a Q tile (IS_K = false) or of K - mu (IS_K = true, mu = the
 // stage's per-channel values): thread ct takes the 16-channel block ct mod
 // (d/16) of every (256 / (d/16))-th row.  Codes of valid rows into codes_blk
 // (row r at codes_blk + r d/2); the scale of every row (0 for rows past
 // `rows`) into the tile's scale-factor blocks sf_tile.
-template <typename T, int D, bool IS_K>
+//
+// MX = true: the MXFP4 variant; the thread pair ct, ct ^ 1 holds the two
+// 16-channel halves of a 32-channel block and shares its maximum by a shuffle.
+template <typename T, int D, bool IS_K, bool MX = false>
 __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const float *mu_s, const float2 *recip,
                                                 uint8_t *codes_blk, uint8_t *sf_tile, uint64_t *empty) {
   constexpr int BPR = D / 16;                      // blocks per row
@@ -175,16 +219,27 @@ __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const f
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = __fsub_rn(v[i], mu[i]);
     }
-    uint32_t w[2], bad[2];
-    const uint32_t sc_code = nvfp4_block_fast(v, recip, w, bad);
+    uint32_t w[2];
+    uint32_t sc_code;
+    if constexpr (MX) {
+      float amax = 0.f;
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {                  // values next to an E2M1 rounding boundary
-      for (uint32_t m = bad[k]; m != 0u; m &= m - 1u) {
-        const int nib = (__ffs(m) - 1) >> 2;
-        const int j = 8 * k + nib;
-        float xj = static_cast<float>(tile[r * D + b * 16 + j]);
-        if (IS_K) xj = __fsub_rn(xj, mu_s[b * 16 + j]);
-        w[k] = (w[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
+      for (int i = 0; i < 16; ++i) amax = fmax_nan(amax, fabsf(v[i]));
+      amax = fmax_nan(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // the block's other 16 channels
+      sc_code = mx_scale_code(amax);
+      mxfp4_codes16(v, sc_code, w);
+    } else {
+      uint32_t bad[2];
+      sc_code = nvfp4_block_fast(v, recip, w, bad);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {                // values next to an E2M1 rounding boundary
+        for (uint32_t m = bad[k]; m != 0u; m &= m - 1u) {
+          const int nib = (__ffs(m) - 1) >> 2;
+          const int j = 8 * k + nib;
+          float xj = static_cast<float>(tile[r * D + b * 16 + j]);
+          if (IS_K) xj = __fsub_rn(xj, mu_s[b * 16 + j]);
+          w[k] = (w[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
+        }
       }
     }
     if (r < rows) __stcs(reinterpret_cast<uint2 *>(codes_blk + r * (D / 2) + b * 8), make_uint2(w[0], w[1]));
@@ -199,7 +254,8 @@ __device__ __forceinline__ void nvfp4_rows_tile(const T *tile, int rows, const f
 // channel pair 2 l, 2 l + 1 of that half, read as one 32-bit word per token
 // (a warp reads 128 consecutive bytes of a row), and stores 16 code bytes
 // per channel.
-template <typename T, int D>
+// MX = true: the MXFP4 variant, one block of 32 tokens per (warp, channel).
+template <typename T, int D, bool MX = false>
 __device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, int Nv, const float2 *recip,
                                              uint8_t *vt_h, uint8_t *sf_tile, uint64_t *empty) {
   constexpr int NCH = D / 64;
@@ -220,20 +276,33 @@ __device__ __forceinline__ void nvfp4_v_tile(const T *tile, int rows, int tok0, 
 #pragma unroll
     for (int ch = 0; ch < 2; ++ch) {
       uint32_t w[4];
+      uint32_t mx_code = 0u;
+      if constexpr (MX) {
+        float amax = 0.f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) amax = fmax_nan(amax, fabsf(x[ch][t]));
+        mx_code = mx_scale_code(amax);
+      }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float blk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) blk[i] = x[ch][16 * h + i];
-        uint32_t wh[2], bad[2];
-        const uint32_t sc_code = nvfp4_block_fast(blk, recip, wh, bad);
+        uint32_t wh[2];
+        uint32_t sc_code = mx_code;
+        if constexpr (MX) {
+          mxfp4_codes16(blk, sc_code, wh);
+        } else {
+          uint32_t bad[2];
+          sc_code = nvfp4_block_fast(blk, recip, wh, bad);
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {              // values next to an E2M1 rounding boundary
-          for (uint32_t m = bad[k]; m != 0u; m &= m - 1u) {
-            const int nib = (__ffs(m) - 1) >> 2;
-            const int r = tg * 32 + 16 * h + 8 * k + nib;
-            const float xj = r < rows ? static_cast<float>(tile[r * D + c + ch]) : 0.f;
-            wh[k] = (wh[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
+          for (int k = 0; k < 2; ++k) {            // values next to an E2M1 rounding boundary
+            for (uint32_t m = bad[k]; m != 0u; m &= m - 1u) {
+              const int nib = (__ffs(m) - 1) >> 2;
+              const int r = tg * 32 + 16 * h + 8 * k + nib;
+              const float xj = r < rows ? static_cast<float>(tile[r * D + c + ch]) : 0.f;
+              wh[k] = (wh[k] & ~(0xFu << (4 * nib))) | (nvfp4_code(xj, sc_code) << (4 * nib));
+            }
           }
         }
         w[2 * h] = wh[0];

@@ -33,7 +33,7 @@ int base_mode(int mode) { return mode & ~kFlagBits; }
 
 bool valid_mode(int mode) {
   const int base = base_mode(mode);
-  return (mode & ~(kFlagBits | 0xFF)) == 0 && (base == SATTN_I8QK_F8PV || base == SATTN_NVFP4);
+  return (mode & ~(kFlagBits | 0xFF)) == 0 && (base == SATTN_I8QK_F8PV || base == SATTN_NVFP4 || base == SATTN_MXFP4);
 }
 
 bool q_per_token(int mode) { return (mode & SATTN_Q_PER_TOKEN) != 0; }
@@ -50,7 +50,9 @@ int check_shape(int B, int H, int N, int d, int mode) {
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool is_nvfp4(int mode) { return base_mode(mode) == SATTN_NVFP4; }
+// The FP4 modes (NVFP4 and MXFP4) share the workspace layout and the kernels.
+bool is_nvfp4(int mode) { return base_mode(mode) == SATTN_NVFP4 || base_mode(mode) == SATTN_MXFP4; }
+bool is_mxfp4(int mode) { return base_mode(mode) == SATTN_MXFP4; }
 
 // The vmax section holds vmax[BH][d] and then the quantiser's work counters:
 // done[2][BH] (K, V statistics) and the ticket counter.  Offset of done from
@@ -173,7 +175,7 @@ template <typename T, int D, int SCHEME>
 int launch_quant(const void *q, const void *k, const void *v, int BH, int N, uint8_t *ws, const sattn_ws_layout_t &L,
                  cudaStream_t st) {
   if (cudaMemsetAsync(ws + L.ksum, 0, L.total - L.ksum, st) != cudaSuccess) return SATTN_ERR_CUDA;
-  if (SCHEME == kSchemeNvfp4 &&
+  if (fp4_scheme(SCHEME) &&
       cudaMemsetAsync(ws + L.sv, 0, static_cast<size_t>(BH) * L.nblk * 1024, st) != cudaSuccess)
     return SATTN_ERR_CUDA;
   const int sms = sm_count();
@@ -216,7 +218,7 @@ int launch_quant(const void *q, const void *k, const void *v, int BH, int N, uin
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL, typename OutT, bool SPARSE>
+template <int D, bool CAUSAL, typename OutT, bool SPARSE, bool MX>
 int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
                       const uint8_t *block_mask, cudaStream_t st) {
   using SL = AttnF4Smem<D>;
@@ -231,7 +233,7 @@ int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, 
   // More than half of the SM's shared memory: one CTA (and its 512 TMEM
   // columns) per SM.
   const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
-  auto kern = attn_nvfp4_kernel<D, CAUSAL, OutT, SPARSE>;
+  auto kern = attn_nvfp4_kernel<D, CAUSAL, OutT, SPARSE, MX>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SATTN_ERR_CUDA;
   AttnF4Args a;
@@ -289,12 +291,19 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
 template <int D, typename OutT>
 int dispatch_attn(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, int causal, float sm,
                   int mode, const uint8_t *mask, cudaStream_t st) {
+  if (is_mxfp4(mode)) {
+    if (mask != nullptr)
+      return causal ? launch_attn_nvfp4<D, true, OutT, true, true>(ws, L, out, BH, N, sm, mask, st)
+                    : launch_attn_nvfp4<D, false, OutT, true, true>(ws, L, out, BH, N, sm, mask, st);
+    return causal ? launch_attn_nvfp4<D, true, OutT, false, true>(ws, L, out, BH, N, sm, nullptr, st)
+                  : launch_attn_nvfp4<D, false, OutT, false, true>(ws, L, out, BH, N, sm, nullptr, st);
+  }
   if (is_nvfp4(mode)) {
     if (mask != nullptr)
-      return causal ? launch_attn_nvfp4<D, true, OutT, true>(ws, L, out, BH, N, sm, mask, st)
-                    : launch_attn_nvfp4<D, false, OutT, true>(ws, L, out, BH, N, sm, mask, st);
-    return causal ? launch_attn_nvfp4<D, true, OutT, false>(ws, L, out, BH, N, sm, nullptr, st)
-                  : launch_attn_nvfp4<D, false, OutT, false>(ws, L, out, BH, N, sm, nullptr, st);
+      return causal ? launch_attn_nvfp4<D, true, OutT, true, false>(ws, L, out, BH, N, sm, mask, st)
+                    : launch_attn_nvfp4<D, false, OutT, true, false>(ws, L, out, BH, N, sm, mask, st);
+    return causal ? launch_attn_nvfp4<D, true, OutT, false, false>(ws, L, out, BH, N, sm, nullptr, st)
+                  : launch_attn_nvfp4<D, false, OutT, false, false>(ws, L, out, BH, N, sm, nullptr, st);
   }
   const bool pt = q_per_token(mode);
   if (mask != nullptr)
@@ -375,6 +384,13 @@ int sattn_quantize(const void *q, const void *k, const void *v, int B, int H, in
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const int BH = B * H;
   const bool fp16 = (mode & SATTN_FP16_IO) != 0;
+  if (is_mxfp4(mode)) {
+    if (d == 128)
+      return fp16 ? launch_quant<__half, 128, kSchemeMxfp4>(q, k, v, BH, N, ws, L, cs)
+                  : launch_quant<__nv_bfloat16, 128, kSchemeMxfp4>(q, k, v, BH, N, ws, L, cs);
+    return fp16 ? launch_quant<__half, 64, kSchemeMxfp4>(q, k, v, BH, N, ws, L, cs)
+                : launch_quant<__nv_bfloat16, 64, kSchemeMxfp4>(q, k, v, BH, N, ws, L, cs);
+  }
   if (is_nvfp4(mode)) {
     if (d == 128)
       return fp16 ? launch_quant<__half, 128, kSchemeNvfp4>(q, k, v, BH, N, ws, L, cs)

@@ -27,6 +27,14 @@
  *                     then NVFP4).  P.V is flushed into the outer
  *                     accumulator every key block, since the stage-1 scale
  *                     changes per block.
+ *   SATTN_MXFP4     : the MXFP4 ablation of SATTN_NVFP4 (same tag page, FP4
+ *                     bullet [15], which reports NVFP4 more accurate than
+ *                     MXFP4): every FP4 operand (Q, K, V, and P's second
+ *                     stage) in blocks of 32 values with one E8M0 scale
+ *                     2^(floor(log2 max|x|) - 2) (OCP Microscaling); the
+ *                     same kernels, tensor layout and workspace layout as
+ *                     SATTN_NVFP4, the E8M0 scale stored for each 16-value
+ *                     half of its block.
  *
  * Tensor layout (all modes): q, k, v, out are contiguous [B, H, N, d] ("BHND"),
  * element type bf16 (default) or fp16 (mode | SATTN_FP16_IO); out has the
@@ -59,12 +67,13 @@ typedef struct CUstream_st *sattn_stream_t;
 typedef enum {
   SATTN_I8QK_F8PV = 0,
   SATTN_NVFP4 = 1,
+  SATTN_MXFP4 = 2,          /* the MXFP4 ablation of SATTN_NVFP4 (above) */
   SATTN_FP16_IO = 0x100,    /* flag: q, k, v, out are fp16 instead of bf16 */
   SATTN_Q_PER_TOKEN = 0x200 /* flag, I8QK_F8PV only: one INT8 scale per query
                                token instead of per 128-token block (the
                                "thread-level quantization" of the QbitAI
                                reprint, txrjy.com, SageAttention paragraph);
-                               NVFP4 with it is SATTN_ERR_UNSUPPORTED */
+                               NVFP4 or MXFP4 with it is SATTN_ERR_UNSUPPORTED */
 } sattn_mode_t;
 
 /* Lazy reference-max threshold of the I8QK_F8PV softmax (powers of two): a
@@ -96,7 +105,9 @@ size_t sattn_workspace_bytes(int B, int H, int N, int d, int mode);
  * summary, bullet [17]: per-block INT8), per-channel FP8 codes and scales of V
  * (explainer, section 1: PV in FP8; V stored transposed, tokens contiguous).
  * NVFP4: E2M1 codes with one E4M3 scale per 16 values of Q, K - mean (along
- * channels) and V (along tokens) (tag page, bullet [15]).  A NaN input makes
+ * channels) and V (along tokens) (tag page, bullet [15]).  MXFP4: E2M1 codes
+ * with one E8M0 scale per 32 values, along the same axes (the ablation of the
+ * same bullet).  A NaN input makes
  * the scale it feeds NaN.  Asynchronous on `stream`: one memset of the
  * workspace's scratch section and one kernel launch, whose tiles of K and V
  * wait (bounded; on time-out the device error word records it, see
@@ -115,7 +126,8 @@ int sattn_quantize(const void *q, const void *k, const void *v,
  * blocks (TurboDiffusion explainer, section 1: INT8 QK, FP8 PV, two-level
  * accumulation).  NVFP4: block-scaled FP4 tensor cores for both products, P
  * quantized in two stages (tag page, SageAttention3 summary, bullets
- * [15][16]).  `out` must not alias the workspace (SATTN_ERR_INVALID_ARG).
+ * [15][16]); MXFP4 the same with E8M0 scales per 32 values, P's second
+ * stage included.  `out` must not alias the workspace (SATTN_ERR_INVALID_ARG).
  * Asynchronous on `stream`. */
 int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out,
                         int B, int H, int N, int d, int causal, float sm_scale,
@@ -260,7 +272,10 @@ int sattn_device_error(int clear);
  *                        block b at byte 16*(m%32) + 4*(m/32) + b
  *              sv E4M3 block scales of V [B*H, ceil(N/128), 2, 512]; same
  *                        byte order with m = channel and b = 16-token block
- *              mu float32 [B*H, d]; ksum, vmax scratch as above */
+ *              mu float32 [B*H, d]; ksum, vmax scratch as above
+ *   MXFP4: as NVFP4, with E8M0 scale codes (scale 2^(code - 127)) of blocks
+ *              of 32 values, each written at both of its 16-value positions
+ *              b = 2c, 2c + 1 of block c */
 typedef struct {
   size_t q8, k8, vt8, sq, sk, sv, mu, ksum, vmax, total;
   int nv, nblk;

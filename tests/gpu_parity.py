@@ -10,7 +10,7 @@ Two criteria, as the accuracy bar of this path states them:
     (max |err| and mean |err|), and the GPU's cosine to exact attention within
     ``COS_TRACK`` of the emulation's (the GPU reproduces the scheme's accuracy);
   * cosine similarity to exact float64 attention >= the bar (0.999 for
-    I8QK_F8PV, 0.995 for NVFP4).  Where the scheme itself (its emulation) is
+    I8QK_F8PV, 0.995 for NVFP4 and its MXFP4 ablation).  Where the scheme itself (its emulation) is
     below the bar on an input, the cosine test of that input is a strict
     expected failure carrying the emulation's measured cosine.
 """
@@ -26,7 +26,7 @@ import bit_quantized_attention_smooth_b200 as sattn
 from oracle import attention as A
 import workloads as W
 
-TOL = {"i8f8": (2e-2, 2e-3, 0.999), "nvfp4": (6e-2, 6e-3, 0.995)}
+TOL = {"i8f8": (2e-2, 2e-3, 0.999), "nvfp4": (6e-2, 6e-3, 0.995), "mxfp4": (6e-2, 6e-3, 0.995)}
 COS_TRACK = 1e-3
 
 
@@ -73,7 +73,7 @@ def run_case(case: Case, mode: str):
         emu = A.attn_quant_emul_i8f8(qf, kf, vf, causal=case.causal, rows=rows,
                                      block_q=1 if case.q_per_token else 128, tau=sattn.I8F8_LAZY_TAU)
     else:
-        emu = A.attn_quant_emul_nvfp4(qf, kf, vf, causal=case.causal, rows=rows)
+        emu = A.attn_quant_emul_nvfp4(qf, kf, vf, causal=case.causal, rows=rows, fmt=mode)
     exact = A.attn_exact(qf, kf, vf, causal=case.causal, rows=rows)
     err = np.abs(got - emu)
     res = dict(finite=bool(np.isfinite(got).all()), err_max=float(err.max()), err_mean=float(err.mean()),

@@ -56,6 +56,16 @@ def test_nvfp4_workspace_layout(L):
     assert lay["total"] == L.sattn_workspace_bytes(1, 12, 32760, 128, NVFP4)
 
 
+def test_mxfp4_mode_shares_the_nvfp4_layout(L):
+    for shape in ((1, 12, 32760, 128), (2, 3, 300, 64)):
+        assert sattn.workspace_layout(*shape, mode="mxfp4") == sattn.workspace_layout(*shape, mode="nvfp4")
+    assert L.sattn_workspace_bytes(1, 2, 256, 64, 2) == L.sattn_workspace_bytes(1, 2, 256, 64, NVFP4) > 0
+    assert L.sattn_workspace_bytes(1, 2, 256, 64, 2 | 0x200) == 0   # per-token Q is I8QK_F8PV only
+    p = ctypes.c_void_p(1 << 20)
+    assert L.sattn_quantize(p, p, p, 1, 2, 256, 64, 2 | 0x200, ctypes.c_void_p(1 << 21), 1 << 30,
+                            None) == UNSUPPORTED
+
+
 def test_workspace_bytes_and_layout(L):
     assert L.sattn_workspace_bytes(1, 2, 256, 64, FP16) > 0
     assert L.sattn_workspace_bytes(1, 2, 0, 64, BF16) == 0       # N < 1
