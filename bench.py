@@ -215,9 +215,10 @@ class ModeRunner:
     """One mode on one set of device inputs: its workspace, device-timed steps
     (quantize + attention, L2 flushed before each) and an accuracy sample."""
 
-    def __init__(self, sattn, q, k, v, causal, mode, q_per_token, flush):
+    def __init__(self, sattn, q, k, v, causal, mode, q_per_token, flush, p_per_token=False):
         self.sattn, self.q, self.k, self.v = sattn, q, k, v
         self.causal, self.mode, self.qtok, self.flush = causal, mode, q_per_token, flush
+        self.ptok = p_per_token
         B, H, N, d = q.shape
         self.shape = (B, H, N, d)
         self.ws = torch.empty(sattn.workspace_bytes(B, H, N, d, mode=mode, dtype=q.dtype, q_per_token=q_per_token),
@@ -230,7 +231,7 @@ class ModeRunner:
         mid = torch.cuda.Event(enable_timing=True)
         mid.record(stream)
         s.fwd_quantized(self.ws, self.shape, causal=self.causal, mode=self.mode, dtype=self.q.dtype, out=self.out,
-                        q_per_token=self.qtok)
+                        q_per_token=self.qtok, p_per_token=self.ptok)
         return mid
 
     def timed(self, n, stream):
@@ -384,11 +385,13 @@ def run_gpu(args):
 
     # the other mode on the same inputs, and per-token Q scales (I8QK_F8PV), beside the headline
     legs = {}
-    for name, (m, qtok) in {"nvfp4": ("nvfp4", False), "i8f8": ("i8f8", False),
-                            "i8f8_q_per_token": ("i8f8", True), "mxfp4": ("mxfp4", False)}.items():
-        if m == mode and qtok == args.q_per_token:
+    for name, (m, qtok, ptok) in {"nvfp4": ("nvfp4", False, False), "i8f8": ("i8f8", False, False),
+                                  "i8f8_q_per_token": ("i8f8", True, False),
+                                  "i8f8_p_per_token": ("i8f8", False, True),
+                                  "mxfp4": ("mxfp4", False, False)}.items():
+        if m == mode and qtok == args.q_per_token and not ptok:
             continue
-        r = ModeRunner(sattn, q, k, v, causal, m, qtok, flush)
+        r = ModeRunner(sattn, q, k, v, causal, m, qtok, flush, p_per_token=ptok)
         r.warm(args.warmup, stream)
         o_step, o_attn, o_quant = r.timed(args.steps, stream)
         legs[name] = {"ms_per_step": median(o_step), "quantize_ms": median(o_quant),

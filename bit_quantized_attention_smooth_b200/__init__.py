@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libsattn.so")
 MODES = {"i8f8": 0, "nvfp4": 1, "mxfp4": 2}
 FP16_IO = 0x100
 Q_PER_TOKEN = 0x200
+P_PER_TOKEN = 0x400
 # Lazy reference-max threshold of the I8QK_F8PV kernel (SATTN_I8F8_LAZY_TAU in
 # include/sattn.h): the row max moves only when a key tile exceeds it by more
 # than this many powers of two, and P's static FP8 scale is 448 * 2^-tau.
@@ -89,12 +90,13 @@ def lib():
     return _lib
 
 
-def mode_code(mode, dtype, q_per_token=False):
+def mode_code(mode, dtype, q_per_token=False, p_per_token=False):
     if mode not in MODES:
         raise ValueError(f"mode must be one of {list(MODES)}")
     if dtype not in (torch.bfloat16, torch.float16):
         raise TypeError("q, k, v must be bfloat16 or float16")
-    return MODES[mode] | (FP16_IO if dtype == torch.float16 else 0) | (Q_PER_TOKEN if q_per_token else 0)
+    return (MODES[mode] | (FP16_IO if dtype == torch.float16 else 0) | (Q_PER_TOKEN if q_per_token else 0) |
+            (P_PER_TOKEN if p_per_token else 0))
 
 
 def _check(status, what):
@@ -148,26 +150,28 @@ def quantize(q, k, v, mode="i8f8", workspace=None, stream=None, q_per_token=Fals
 
 
 def fwd_quantized(workspace, shape, causal=False, sm_scale=None, mode="i8f8", dtype=torch.bfloat16,
-                  out=None, stream=None, q_per_token=False):
-    """Attention over a workspace filled by ``quantize``; returns out [B, H, N, d]."""
+                  out=None, stream=None, q_per_token=False, p_per_token=False):
+    """Attention over a workspace filled by ``quantize``; returns out [B, H, N, d].
+    ``p_per_token``: P quantised per query row and key block (I8QK_F8PV only)."""
     B, H, N, d = shape
     if out is None:
         out = torch.empty((B, H, N, d), dtype=dtype, device=workspace.device)
     _check(lib().sattn_fwd_quantized(workspace.data_ptr(), workspace.numel(), out.data_ptr(),
                                      B, H, N, d, int(bool(causal)), float(sm_scale or 0.0),
-                                     mode_code(mode, dtype, q_per_token), _stream(stream)),
+                                     mode_code(mode, dtype, q_per_token, p_per_token), _stream(stream)),
            "sattn_fwd_quantized")
     return out
 
 
-def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None, q_per_token=False):
+def fwd(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream=None, q_per_token=False,
+        p_per_token=False):
     """O = softmax(Q K^T * sm_scale) V with quantised operands (library-owned workspace)."""
     B, H, N, d = _check_qkv(q, k, v)
     if out is None:
         out = torch.empty_like(q)
     _check(lib().sattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, H, N, d,
-                           int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype, q_per_token),
-                           _stream(stream)),
+                           int(bool(causal)), float(sm_scale or 0.0),
+                           mode_code(mode, q.dtype, q_per_token, p_per_token), _stream(stream)),
            "sattn_fwd")
     return out
 

@@ -28,6 +28,11 @@
 //   O = (O_out + O_in) * s_v[c] / (c_P l).
 // Q scales: one per 128-token tile, or one per token (the row's thread holds
 // its own scale, so the finer granularity costs nothing here).
+// Per-token P (PTOK, the 8-bit bullet [17] of the SageAttention tag page): P
+// is quantised against each row's maximum within the key tile, p8 =
+// E4M3(448 2^(S2 - m_tile)), and the tile's P V is added into O_out with the
+// factor 2^(m_tile - m) (m = the exact running max); each tile takes a max
+// pass and a P pass over S, and O_in is flushed after every tile.
 //
 // CTA = two 128-row query tiles (A, B) of one (b, h) sharing every K/V tile;
 // 12 warps in 3 warpgroups:
@@ -230,7 +235,31 @@ __device__ __forceinline__ float p_pass(uint32_t s_tmem, float c, float b, uint8
   return tsum2.x + tsum2.y;
 }
 
-template <int D, bool CAUSAL, typename OutT, bool SPARSE>
+// Largest valid INT8 score of the row in an S tile (masked keys read as
+// kMaskedScore = INT_MIN, so a row without a valid key returns INT_MIN).
+template <int W>
+__device__ __forceinline__ int s_max_pass(uint32_t s_tmem, bool masked, int kv0, int N, bool causal, int row_g) {
+  static_assert(W == 32 || W == 64, "columns per TMEM round trip");
+  int mx = static_cast<int>(kMaskedScore);
+#pragma unroll 1
+  for (int hh = 0; hh < kTile / W; ++hh) {
+    uint32_t s0[32], s1[32];
+    tmem_ld_32x32b_x32(s_tmem + hh * W, s0);
+    if constexpr (W == 64) tmem_ld_32x32b_x32(s_tmem + hh * W + 32, s1);
+    tmem_ld_wait(s0);
+    if constexpr (W == 64) tmem_ld_wait(s1);
+    if (masked) {
+      mask_chunk(s0, kv0 + hh * W, N, causal, row_g);
+      if constexpr (W == 64) mask_chunk(s1, kv0 + hh * W + 32, N, causal, row_g);
+    }
+    mx = max(mx, tree_max32(s0));
+    if constexpr (W == 64) mx = max(mx, tree_max32(s1));
+  }
+  return mx;
+}
+
+// PTOK = true: per-token P (see the file comment).
+template <int D, bool CAUSAL, typename OutT, bool SPARSE, bool PTOK = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_i8f8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
@@ -413,7 +442,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ok = ok && mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t acc = (t % kFlushEvery) != 0 ? 1u : 0u;
+            const uint32_t acc = (!PTOK && (t % kFlushEvery) != 0) ? 1u : 0u;   // PTOK: one tile per O_in
             const uint32_t sP = smem_u32(smem + L::kP + pb * L::kPBytes);
             const uint32_t sV = smem_u32(smem + L::kV + s * L::kVBytes);
 #pragma unroll
@@ -463,6 +492,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float m_ref = -INFINITY;   // reference max of the row (lazy)
     float lsum = 0.f;          // sum of c_P * P~ (the static FP8 scale folded in)
     float beta = 1.f;          // the outer accumulator is beta * o_out (rescaled lazily)
+    float f_pend = 1.f;        // PTOK: factor of the tile whose P V is pending, 2^(m_tile - m)
     bool ok = true;
 
     int n = 0;                 // key tiles processed (the S, P and O_in barriers advance per tile)
@@ -479,36 +509,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int pb = x * 2 + (n & 1);
       if (!mbar_wait(&pv_done[pb], ((n >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
       uint8_t *prow = p_base + (n & 1) * L::kPBytes;
-      // speculative pass with the current reference max (0 at the first tile,
-      // which only serves to find the tile's row max)
-      const float m_try = n > 0 ? m_ref : 0.f;
       float2 xm2 = make_float2(-INFINITY, -INFINITY);
-      float tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_try - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
-      // x = S2 - m + log2 c_P;  the row max moves when S2max - m > tau  <=>  xmax > log2 448
-      const float xmax = fmaxf(xm2.x, xm2.y);
-      const bool up = n == 0 || xmax > kLog2_448;
-      const bool moved = __any_sync(0xffffffffu, up);   // warp-uniform
-      float m_new = m_ref, alpha = 1.f;
-      if (moved) {
-        if (up) m_new = fmaxf(m_ref, xmax + (m_try - kLog2_CP));   // the tile's row max
-        alpha = n > 0 ? ex2_approx(m_ref - m_new) : 0.f;
-        tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_new - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
+      float tsum, m_new = m_ref, alpha = 1.f, f_tile = 1.f;
+      bool moved = false;
+      if constexpr (PTOK) {
+        // per-token P: the tile's row max first, then the codes of 448 2^(S2 - m_tile)
+        const int smax = s_max_pass<CAUSAL ? 32 : 64>(s_tmem, masked, kv0, N, CAUSAL, row_g);
+        const float m_tile = smax != static_cast<int>(kMaskedScore) ? static_cast<float>(smax) * c : -INFINITY;
+        // a row without a valid key in the tile (all masked) writes zero codes
+        tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_tile != -INFINITY ? m_tile - kLog2_448 : 0.f, prow, r, masked,
+                                        kv0, N, CAUSAL, row_g, xm2);
+        m_new = fmaxf(m_ref, m_tile);
+        if (m_new == -INFINITY) {                     // no valid key in the row so far
+          alpha = 1.f;
+          f_tile = 0.f;
+        } else {
+          alpha = n > 0 ? ex2_approx(m_ref - m_new) : 0.f;
+          f_tile = ex2_approx(m_tile - m_new);
+        }
+        tsum *= f_tile;
+      } else {
+        // speculative pass with the current reference max (0 at the first tile,
+        // which only serves to find the tile's row max)
+        const float m_try = n > 0 ? m_ref : 0.f;
+        tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_try - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
+        // x = S2 - m + log2 c_P;  the row max moves when S2max - m > tau  <=>  xmax > log2 448
+        const float xmax = fmaxf(xm2.x, xm2.y);
+        const bool up = n == 0 || xmax > kLog2_448;
+        moved = __any_sync(0xffffffffu, up);   // warp-uniform
+        if (moved) {
+          if (up) m_new = fmaxf(m_ref, xmax + (m_try - kLog2_CP));   // the tile's row max
+          alpha = n > 0 ? ex2_approx(m_ref - m_new) : 0.f;
+          tsum = p_pass<CAUSAL ? 32 : 64>(s_tmem, c, m_new - kLog2_CP, prow, r, masked, kv0, N, CAUSAL, row_g, xm2);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[x]);
       lsum = fmaf(alpha, lsum, tsum);
 
-      // two-level accumulation: flush O_in at a group start, or rescale when the reference max moved
-      const bool boundary = n > 0 && (n % kFlushEvery) == 0;
-      const bool grow = n > 0 && moved;
+      // two-level accumulation: flush O_in at a group start (PTOK: after every
+      // tile, with its factor), or rescale when the reference max moved
+      const bool boundary = n > 0 && (PTOK || (n % kFlushEvery) == 0);
+      const bool grow = !PTOK && n > 0 && moved;
       if (boundary || grow) {
         const int t = n - 1;
         if (!mbar_wait(&pv_done[x * 2 + (t & 1)], (t >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (boundary) {
-          // O_out += O_in (both relative to m_ref); o_out holds O_out / beta
-          const float inv_beta = 1.f / beta;
+          // O_out += O_in (both relative to m_ref; PTOK: O_in times its tile's
+          // factor); o_out holds O_out / beta
+          const float inv_beta = PTOK ? f_pend / beta : 1.f / beta;
 #pragma unroll
           for (int ch = 0; ch < D / 32; ch += 2) {
             uint32_t o0[32], o1[32];
@@ -554,6 +605,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[pb]);
       m_ref = m_new;
+      f_pend = f_tile;
       ++n;
     }
 
@@ -573,8 +625,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float o0 = fmaf(beta, o_out[ch * 32 + i], __uint_as_float(o[i])) * sv[ch * 32 + i] * inv_l;
-            const float o1 = fmaf(beta, o_out[ch * 32 + i + 1], __uint_as_float(o[i + 1])) * sv[ch * 32 + i + 1] * inv_l;
+            const float i0 = PTOK ? f_pend * __uint_as_float(o[i]) : __uint_as_float(o[i]);
+            const float i1 = PTOK ? f_pend * __uint_as_float(o[i + 1]) : __uint_as_float(o[i + 1]);
+            const float o0 = fmaf(beta, o_out[ch * 32 + i], i0) * sv[ch * 32 + i] * inv_l;
+            const float o1 = fmaf(beta, o_out[ch * 32 + i + 1], i1) * sv[ch * 32 + i + 1] * inv_l;
             packed[i >> 1] = pack2_out<OutT>(o0, o1);
           }
           if (row_g < N) {

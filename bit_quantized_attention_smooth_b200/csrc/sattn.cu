@@ -27,7 +27,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Kernels this library has launched since load (or the last reset).
 std::atomic<unsigned long long> g_launches{0};
 
-constexpr int kFlagBits = SATTN_FP16_IO | SATTN_Q_PER_TOKEN;
+constexpr int kFlagBits = SATTN_FP16_IO | SATTN_Q_PER_TOKEN | SATTN_P_PER_TOKEN;
 
 int base_mode(int mode) { return mode & ~kFlagBits; }
 
@@ -37,11 +37,12 @@ bool valid_mode(int mode) {
 }
 
 bool q_per_token(int mode) { return (mode & SATTN_Q_PER_TOKEN) != 0; }
+bool p_per_token(int mode) { return (mode & SATTN_P_PER_TOKEN) != 0; }
 
 int check_shape(int B, int H, int N, int d, int mode) {
   if (B < 1 || H < 1 || N < 1) return SATTN_ERR_INVALID_ARG;
   if (!valid_mode(mode)) return SATTN_ERR_INVALID_ARG;
-  if (q_per_token(mode) && base_mode(mode) != SATTN_I8QK_F8PV) return SATTN_ERR_UNSUPPORTED;
+  if ((q_per_token(mode) || p_per_token(mode)) && base_mode(mode) != SATTN_I8QK_F8PV) return SATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return SATTN_ERR_UNSUPPORTED;
   const long long total = static_cast<long long>(B) * H * N * d;
   if (total >= (1LL << 31) || static_cast<long long>(B) * H >= 65536) return SATTN_ERR_UNSUPPORTED;
@@ -250,7 +251,7 @@ int launch_attn_nvfp4(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, 
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL, typename OutT, bool SPARSE>
+template <int D, bool CAUSAL, typename OutT, bool SPARSE, bool PTOK>
 int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int BH, int N, float sm_scale,
                      bool per_token, const uint8_t *block_mask, cudaStream_t st) {
   using SL = AttnSmem<D>;
@@ -264,7 +265,7 @@ int launch_attn_i8f8(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, i
   // More than half of the SM's shared memory: one CTA (and its 512 TMEM
   // columns) per SM.
   const int smem = SL::kAlloc > 118 * 1024 ? SL::kAlloc : 118 * 1024;
-  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, SPARSE>;
+  auto kern = attn_i8f8_kernel<D, CAUSAL, OutT, SPARSE, PTOK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return SATTN_ERR_CUDA;
   // The kernel's setmaxnreg split must fit in its launch registers, or its
@@ -306,11 +307,16 @@ int dispatch_attn(const uint8_t *ws, const sattn_ws_layout_t &L, void *out, int 
                   : launch_attn_nvfp4<D, false, OutT, false, false>(ws, L, out, BH, N, sm, nullptr, st);
   }
   const bool pt = q_per_token(mode);
+  if (p_per_token(mode)) {
+    if (mask != nullptr) return SATTN_ERR_UNSUPPORTED;   // per-token P: dense calls only
+    return causal ? launch_attn_i8f8<D, true, OutT, false, true>(ws, L, out, BH, N, sm, pt, nullptr, st)
+                  : launch_attn_i8f8<D, false, OutT, false, true>(ws, L, out, BH, N, sm, pt, nullptr, st);
+  }
   if (mask != nullptr)
-    return causal ? launch_attn_i8f8<D, true, OutT, true>(ws, L, out, BH, N, sm, pt, mask, st)
-                  : launch_attn_i8f8<D, false, OutT, true>(ws, L, out, BH, N, sm, pt, mask, st);
-  return causal ? launch_attn_i8f8<D, true, OutT, false>(ws, L, out, BH, N, sm, pt, nullptr, st)
-                : launch_attn_i8f8<D, false, OutT, false>(ws, L, out, BH, N, sm, pt, nullptr, st);
+    return causal ? launch_attn_i8f8<D, true, OutT, true, false>(ws, L, out, BH, N, sm, pt, mask, st)
+                  : launch_attn_i8f8<D, false, OutT, true, false>(ws, L, out, BH, N, sm, pt, mask, st);
+  return causal ? launch_attn_i8f8<D, true, OutT, false, false>(ws, L, out, BH, N, sm, pt, nullptr, st)
+                : launch_attn_i8f8<D, false, OutT, false, false>(ws, L, out, BH, N, sm, pt, nullptr, st);
 }
 
 // Checks of a block-sparse call beyond those of the dense one.

@@ -69,11 +69,22 @@ typedef enum {
   SATTN_NVFP4 = 1,
   SATTN_MXFP4 = 2,          /* the MXFP4 ablation of SATTN_NVFP4 (above) */
   SATTN_FP16_IO = 0x100,    /* flag: q, k, v, out are fp16 instead of bf16 */
-  SATTN_Q_PER_TOKEN = 0x200 /* flag, I8QK_F8PV only: one INT8 scale per query
+  SATTN_Q_PER_TOKEN = 0x200, /* flag, I8QK_F8PV only: one INT8 scale per query
                                token instead of per 128-token block (the
                                "thread-level quantization" of the QbitAI
                                reprint, txrjy.com, SageAttention paragraph);
                                NVFP4 or MXFP4 with it is SATTN_ERR_UNSUPPORTED */
+  SATTN_P_PER_TOKEN = 0x400  /* flag, I8QK_F8PV only, dense calls only: P
+                               quantized per token (tag page, SageAttention3
+                               summary, 8-bit bullet [17]): each query row's
+                               P of a key block is stored as
+                               E4M3(448 * P~ / rowmax of the block) and the
+                               block's P V is scaled back by that max; the
+                               inner accumulator is then flushed after every
+                               key block.  The quantized operands (and the
+                               workspace) are those of the mode without it.
+                               With another mode, or in a block-sparse call:
+                               SATTN_ERR_UNSUPPORTED */
 } sattn_mode_t;
 
 /* Lazy reference-max threshold of the I8QK_F8PV softmax (powers of two): a

@@ -38,12 +38,13 @@ class Case:
     heads: tuple = None         # sampled (b, h) pairs (None: all)
     via_fwd: bool = False       # sattn_fwd (library workspace) instead of quantize + fwd_quantized
     q_per_token: bool = False
+    p_per_token: bool = False   # I8QK_F8PV: P quantised per query row and key block
     miss: str = None            # the scheme's own cosine is below the bar: why, with the measured value
 
     @property
     def id(self):
         causal = "-causal" if self.causal and not self.w.name.endswith("-causal") else ""
-        return (f"{self.w.name}{causal}{'-qtok' if self.q_per_token else ''}"
+        return (f"{self.w.name}{causal}{'-qtok' if self.q_per_token else ''}{'-ptok' if self.p_per_token else ''}"
                 f"{'-sampled' if self.rows is not None else ''}")
 
 
@@ -57,11 +58,12 @@ def run_case(case: Case, mode: str):
     w = case.w
     q, k, v = W.make_inputs(w, "cuda")
     if case.via_fwd:
-        out = sattn.fwd(q, k, v, causal=case.causal, mode=mode, q_per_token=case.q_per_token)
+        out = sattn.fwd(q, k, v, causal=case.causal, mode=mode, q_per_token=case.q_per_token,
+                        p_per_token=case.p_per_token)
     else:
         ws = sattn.quantize(q, k, v, mode=mode, q_per_token=case.q_per_token)
         out = sattn.fwd_quantized(ws, q.shape, causal=case.causal, mode=mode, dtype=q.dtype,
-                                  q_per_token=case.q_per_token)
+                                  q_per_token=case.q_per_token, p_per_token=case.p_per_token)
     torch.cuda.synchronize()
     heads = list(case.heads) if case.heads is not None else [(b, h) for b in range(w.B) for h in range(w.H)]
     rows = np.arange(w.N) if case.rows is None else np.asarray(case.rows, dtype=np.int64)
@@ -69,7 +71,10 @@ def run_case(case: Case, mode: str):
     del q, k, v, out
     got = np.stack([o[b, h][rows] for (b, h) in heads])
     qf, kf, vf = W.make_heads_f32(w, heads)
-    if mode == "i8f8":
+    if mode == "i8f8" and case.p_per_token:
+        emu = A.attn_quant_emul_i8f8_smooth(qf, kf, vf, causal=case.causal, rows=rows,
+                                            block_q=1 if case.q_per_token else 128, smooth_q=False, p_per_token=True)
+    elif mode == "i8f8":
         emu = A.attn_quant_emul_i8f8(qf, kf, vf, causal=case.causal, rows=rows,
                                      block_q=1 if case.q_per_token else 128, tau=sattn.I8F8_LAZY_TAU)
     else:

@@ -107,7 +107,8 @@ def test_invalid_arguments_rejected_before_launch(L):
     g = L.sattn_fwd
     assert g(p, p, p, None, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID
     assert g(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
-    assert g(p, p, p, mis, 1, 2, 256, 128, 0, 0.0, 0x400, None) == INVALID   # unknown flag
+    assert g(p, p, p, mis, 1, 2, 256, 128, 0, 0.0, 0x800, None) == INVALID   # unknown flag
+    assert g(p, p, p, p, 1, 2, 256, 64, 0, 0.0, NVFP4 | 0x400, None) == UNSUPPORTED   # per-token P: I8QK_F8PV only
 
 
 def test_fwd_host_rejects_bad_arguments_before_any_cuda_call(L):
@@ -119,8 +120,9 @@ def test_fwd_host_rejects_bad_arguments_before_any_cuda_call(L):
     assert h(p, p, p, p, 1, 2, 256, 64, 0, 0.0, BF16, None) == INVALID      # out aliases q
     assert h(p, p, p, o, 1, 2, 256, 96, 0, 0.0, BF16, None) == UNSUPPORTED
     assert h(p, p, p, o, 1, 2, 0, 64, 0, 0.0, BF16, None) == INVALID
-    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, 0x400, None) == INVALID     # unknown flag
+    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, 0x800, None) == INVALID     # unknown flag
     assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, NVFP4 | QTOK, None) == UNSUPPORTED
+    assert h(p, p, p, o, 1, 2, 256, 64, 0, 0.0, NVFP4 | 0x400, None) == UNSUPPORTED   # per-token P
 
 
 def test_fwd_host_binding_rejects_device_or_mismatched_tensors():
@@ -144,7 +146,10 @@ def test_per_token_q_layout(L):
     assert tok["sk"] - tok["sq"] >= 6 * 1000 * 4 > blk["sk"] - blk["sq"]
     assert tok["total"] == L.sattn_workspace_bytes(2, 3, 1000, 128, QTOK)
     assert L.sattn_workspace_bytes(2, 3, 1000, 128, NVFP4 | QTOK) == 0
-    assert L.sattn_workspace_bytes(2, 3, 1000, 128, 0x400) == 0
+    assert L.sattn_workspace_bytes(2, 3, 1000, 128, 0x800) == 0          # unknown flag
+    # per-token P changes the attention, not the quantised operands
+    assert L.sattn_workspace_bytes(2, 3, 1000, 128, 0x400) == L.sattn_workspace_bytes(2, 3, 1000, 128, 0)
+    assert L.sattn_workspace_bytes(2, 3, 1000, 128, NVFP4 | 0x400) == 0
 
 
 def test_block_sparse_entry_points_validate_before_any_cuda_call(L):

@@ -7,6 +7,8 @@ mean |err| <= 2e-3; and with the exact float64 attention by cosine similarity
 >= 0.999.  On the inputs with 0.1 % x20 Q outliers the scheme itself misses
 0.999 (its emulation does), so the cosine test of those inputs is a strict
 expected failure that records the measured value (see tests/gpu_parity.py).
+The per-token Q and per-token P variants are compared in the same way with
+the oracle's emulations of those variants.
 """
 
 import numpy as np
@@ -165,14 +167,50 @@ QTOK_CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", ATTN_CASES + QTOK_CASES, ids=lambda c: c.id)
+# P quantised per query row and key block (the 8-bit bullet [17] of the tag
+# page), compared with the oracle's per-token-P emulation; alone and with
+# per-token Q scales
+PTOK_CASES = [
+    Case(W.SMALL, p_per_token=True),
+    Case(W.custom(1, 2, 17, 64, "fp16", seed=12), causal=True, p_per_token=True),
+    Case(W.custom(1, 3, 129, 128, seed=14), causal=True, p_per_token=True),
+    Case(W.custom(2, 2, 300, 64, seed=15), causal=True, p_per_token=True, q_per_token=True),
+    Case(W.custom(1, 2, 1000, 128, seed=16, q_outlier_frac=1e-3), p_per_token=True,
+         miss=OUTLIERS.format("block", 0.99594)),
+    Case(W.custom(1, 2, 1000, 128, seed=16, q_outlier_frac=1e-3), p_per_token=True, q_per_token=True,
+         miss=OUTLIERS.format("token", 0.99837)),
+    Case(W.custom(1, 2, 1536, 64, "fp16", seed=17), p_per_token=True),
+    Case(W.MID, rows=tuple(np.concatenate([np.arange(0, 4096, 61), [4095]]).tolist()), p_per_token=True,
+         q_per_token=True, miss=OUTLIERS.format("token", 0.99860)),
+    Case(W.VIDEO_32760, rows=sample_rows(32760, 60, 0, (0, 127, 32639, 32759)),
+         heads=((0, 0), (0, 5), (0, 11), (0, 7)), via_fwd=True, p_per_token=True,
+         miss=OUTLIERS.format("block", 0.99765)),
+    Case(W.sweep(128, 2048, True), causal=True, rows=sample_rows(2048, 48, 2048, (0, 2047)),
+         heads=((0, 0), (3, 31), (1, 17)), p_per_token=True),
+]
+
+
+@pytest.mark.parametrize("case", ATTN_CASES + QTOK_CASES + PTOK_CASES, ids=lambda c: c.id)
 def test_attention_matches_oracle(case):
     check_parity(case, "i8f8")
 
 
-@pytest.mark.parametrize("case", miss_params(ATTN_CASES + QTOK_CASES))
+@pytest.mark.parametrize("case", miss_params(ATTN_CASES + QTOK_CASES + PTOK_CASES))
 def test_cosine_bar_where_the_scheme_misses_it(case):
     check_cosine_bar(case, "i8f8")
+
+
+def test_per_token_p_is_rejected_where_unsupported():
+    w = W.custom(1, 2, 300, 64, seed=55)
+    q, k, v = W.make_inputs(w, "cuda")
+    with pytest.raises(sattn.SattnError):
+        sattn.fwd(q, k, v, mode="nvfp4", p_per_token=True)
+    m = torch.ones((1, 2, 3, 3), dtype=torch.uint8, device="cuda")
+    L = sattn.lib()
+    mc = sattn.mode_code("i8f8", q.dtype, p_per_token=True)
+    out = torch.empty_like(q)
+    assert L.sattn_fwd_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), 1, 2, 300, 64, 0, 0.0, mc,
+                              m.data_ptr(), None) == 2   # SATTN_ERR_UNSUPPORTED, nothing launched
 
 
 def _check_attention(w, causal):
