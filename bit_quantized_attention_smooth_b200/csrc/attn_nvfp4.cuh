@@ -75,7 +75,8 @@ struct AttnF4Smem {
   static constexpr int kSfVo = kSfK + kKVStages * kSfQK;
   static constexpr int kSfPo = kSfVo + kKVStages * kSfV;
   static constexpr int kX = kSfPo + 2 * kSfP;          // float [2 phases][4 quarters][128] + [4][128]
-  static constexpr int kMask = kX + (2 * 4 * 128 + 4 * 128) * 4;   // [kMaxMaskTiles] bytes (block-sparse calls)
+  static constexpr int kLsc = kX + (2 * 4 * 128 + 4 * 128) * 4;   // float2 [128]: (value, log2 value) of E4M3 codes
+  static constexpr int kMask = kLsc + 128 * 8;        // [kMaxMaskTiles] bytes (block-sparse calls)
   static constexpr int kBar = kMask + kMaxMaskTiles;
   // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], s_free[2],
   // p_full[2], pv_done[2], quad[4], drain
@@ -223,6 +224,11 @@ __global__ void __launch_bounds__(kF4Threads, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+  }
+  if (!MX && tid < 128) {
+    // every non-negative E4M3 code's value and log2 (the stage-2 scales of P)
+    const float v = e4m3_to_float(static_cast<uint32_t>(tid));
+    reinterpret_cast<float2 *>(smem + L::kLsc)[tid] = make_float2(v, v > 0.f ? __log2f(v) : 0.f);
   }
   tc_fence_before();
   __syncthreads();
@@ -447,13 +453,14 @@ __global__ void __launch_bounds__(kF4Threads, 1)
         const int blk = (kq & 1) * 2 + hb;                // 16-key block within the 64-key slice
         // scale = E4M3(block max of P2 / 6): the division by 6 folds into the exponent
         const float amax6 = ex2_approx(fmaf(bmax[hb], cl, -moff6));
-        const uint32_t sc_code = cvt_e4m3x2(amax6, 0.f) & 0xFFu;
-        const float sc = e4m3_to_float(sc_code);
+        const uint32_t sc_code = cvt_e4m3x2(amax6, 0.f) & 0x7Fu;   // amax6 >= 0: sign bit clear
+        const float2 scl = reinterpret_cast<const float2 *>(smem + L::kLsc)[sc_code];   // scale, log2 scale
+        const float sc = scl.x;
         psf[sf_offset(r, blk)] = static_cast<uint8_t>(sc_code);
         // P2 / scale = 2^(S2 - moff - log2 scale): the division folds into the
         // exponent's constant; the block's P2 sum is scale * sum(P2 / scale).
         const bool live = sc > 0.f;
-        const float lsc = live ? __log2f(sc) : 0.f;
+        const float lsc = scl.y;
         const float2 nb2 = make_float2(-(moff + lsc), -(moff + lsc));
         float2 bsum = make_float2(0.f, 0.f);
         float2 y[8];
