@@ -9,7 +9,7 @@ events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--mode i8f8|nvfp4|mxfp4] [--workload NAME] [--causal] [--q-per-token]
-    python bench.py --sweep [--steps K]      # the B=4 H=32 sweep, both modes
+    python bench.py --sweep [--steps K]      # the B=4 H=32 sweep, all three modes
 
 Prints ONE JSON line on rank 0 (the sweep: one per point and mode).  Step and
 kernel times are medians over the timed steps.  Under torchrun (N > 1) every rank runs its own
@@ -304,7 +304,7 @@ def init_dist():
 
 def run_sweep(args):
     """The B=4, H=32 sweep (d in {64,128}, N in 1024..32768, causal and
-    non-causal), both modes: one JSON line per point and mode.  Inputs follow
+    non-causal), in the three modes: one JSON line per point and mode.  Inputs follow
     the workload recipe but are drawn on the device (a different random stream
     from the CPU recipe the parity tests use), so that 1 GB tensors are made
     in milliseconds."""
@@ -317,7 +317,7 @@ def run_sweep(args):
     for (d, N, causal) in W.SWEEP_POINTS:
         w = W.sweep(d, N, causal)
         q, k, v = W.make_inputs_device(w, dev)
-        for mode in ("i8f8", "nvfp4"):
+        for mode in ("i8f8", "nvfp4", "mxfp4"):
             r = ModeRunner(sattn, q, k, v, causal, mode, False, flush)
             r.warm(args.warmup, stream)
             step_ms, attn_ms, quant_ms = r.timed(args.steps, stream)
@@ -545,7 +545,7 @@ def main():
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--q-per-token", action="store_true", help="I8QK_F8PV with one Q scale per token")
     ap.add_argument("--sweep", action="store_true",
-                    help="time the B=4 H=32 sweep in both modes (one JSON line per point and mode)")
+                    help="time the B=4 H=32 sweep in the three modes (one JSON line per point and mode)")
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps of the GPU path only (for ncu captures)")
     args = ap.parse_args()
