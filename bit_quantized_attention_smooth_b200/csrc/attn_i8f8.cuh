@@ -61,7 +61,7 @@ namespace sattn {
 constexpr int kTile = 128;          // query rows and keys per tile
 constexpr int kQTiles = 2;          // query tiles per CTA
 constexpr int kKVStages = 3;
-constexpr int kFlushEvery = 4;      // G: key tiles per inner accumulation group
+constexpr int kFlushEvery = 8;      // G: key tiles per inner accumulation group
 constexpr int kAttnThreads = 384;       // 3 warpgroups
 constexpr int kSoftmaxRegs = 232;       // per thread, softmax warpgroups 0 and 1
 constexpr int kControlRegs = 40;        // per thread, warpgroup 2 (TMA, MMA, 2 idle warps)
