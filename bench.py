@@ -427,7 +427,7 @@ def run_gpu(args):
         peaks, src = measured_peaks()
         peak = PEAK_RATIO[mode] * peaks["bf16_tflops"]
         att = attention_report(w, mode, causal, attn_med, peaks)
-        achieved = att["tops"]
+        achieved = att["tops"] / (2 if causal else 1)   # algorithmic work: a causal pass does half the pairs
         for name, leg in legs.items():
             m = name if name in ("nvfp4", "mxfp4") else "i8f8"
             leg["attention_kernel"] = attention_report(w, m, causal, leg.pop("attention_kernel_ms"), peaks)
@@ -436,7 +436,8 @@ def run_gpu(args):
         if os.path.exists(tpath):
             with open(tpath) as f:
                 tj = json.load(f)
-            if tj.get("kernel_hash") == kernel_hash(mode) and tj.get("workload") == w.name:
+            # the record is of the dense non-causal kernel on this workload
+            if tj.get("kernel_hash") == kernel_hash(mode) and tj.get("workload") == w.name and not causal:
                 traffic = tj.get("dram_bytes_per_launch_full")
         quant = quantizer_roofline(sattn, w, q, mode, args.q_per_token, median(quant_ms), peaks, src)
         cpu = None
