@@ -539,7 +539,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sattn", choices=["sattn", "reference"])
-    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)   # the two-size fit underestimates large samples
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="i8f8", choices=["i8f8", "nvfp4", "mxfp4"])
     ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(W.WORKLOADS))
