@@ -151,7 +151,8 @@ int sattn_fwd_quantized(const void *workspace, size_t ws_bytes, void *out,
  * Attention, TurboDiffusion explainer, SLA section, with the mask given by
  * the caller).  block_mask: device memory, uint8 [B*H][nblk][nblk], nblk =
  * ceil(N / 128), entry [bh][i][j] nonzero = query block i keeps key block j.
- * A query block that keeps no key block gets zero output rows.  Both modes;
+ * A query block that keeps no key block gets zero output rows.  Every mode
+ * (not with SATTN_P_PER_TOKEN: SATTN_ERR_UNSUPPORTED);
  * nblk <= 2048 (N <= 262144), else SATTN_ERR_UNSUPPORTED; block_mask == NULL
  * is SATTN_ERR_INVALID_ARG.  The
  * mask is read by the kernel, so it must stay unchanged until `stream` has
