@@ -32,7 +32,7 @@ STATUS = {0: "SATTN_OK", 1: "SATTN_ERR_INVALID_ARG", 2: "SATTN_ERR_UNSUPPORTED",
 EXPORTS = ("sattn_workspace_bytes", "sattn_quantize", "sattn_fwd_quantized", "sattn_fwd",
            "sattn_status_string", "sattn_device_error", "sattn_workspace_layout", "sattn_fwd_noalloc",
            "sattn_fwd_host", "sattn_kernel_launches", "sattn_debug_set_wait_limit", "sattn_debug_withhold_statistics",
-           "sattn_fwd_quantized_sparse", "sattn_fwd_sparse")
+           "sattn_fwd_quantized_sparse", "sattn_fwd_sparse", "sattn_debug_scores")
 
 
 class SattnError(RuntimeError):
@@ -86,6 +86,8 @@ def lib():
         L.sattn_fwd_quantized_sparse.argtypes = [vp, sz, vp, i, i, i, i, i, f, i, vp, vp]
         L.sattn_fwd_sparse.restype = i
         L.sattn_fwd_sparse.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, i, vp, vp]
+        L.sattn_debug_scores.restype = i
+        L.sattn_debug_scores.argtypes = [vp, sz, i, i, i, i, i, vp, vp]
         _lib = L
     return _lib
 
@@ -237,6 +239,18 @@ def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream
                                 int(bool(causal)), float(sm_scale or 0.0), mode_code(mode, q.dtype, q_per_token),
                                 _stream(stream)),
            "sattn_fwd_host")
+    return out
+
+
+def debug_scores(workspace, shape, mode="i8f8", dtype=torch.bfloat16, stream=None, q_per_token=False):
+    """Test accessor: the INT8 scores q8 . k8^T of a quantised workspace,
+    int32 [B, H, Np, Np] (Np = N rounded up to 128), computed on the tensor cores."""
+    B, H, N, d = shape
+    np_ = (N + 127) // 128 * 128
+    out = torch.empty((B, H, np_, np_), dtype=torch.int32, device=workspace.device)
+    _check(lib().sattn_debug_scores(workspace.data_ptr(), workspace.numel(), B, H, N, d,
+                                    mode_code(mode, dtype, q_per_token), out.data_ptr(), _stream(stream)),
+           "sattn_debug_scores")
     return out
 
 

@@ -14,6 +14,7 @@
 #include "../../include/sattn.h"
 #include "attn_i8f8.cuh"
 #include "attn_nvfp4.cuh"
+#include "debug_scores.cuh"
 #include "quant_fused.cuh"
 
 namespace sattn {
@@ -641,6 +642,33 @@ int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile) {
       cudaMemcpyToSymbol(g_withhold_k_tile, &withhold_k_tile, sizeof(withhold_k_tile)) != cudaSuccess)
     return SATTN_ERR_CUDA;
   return SATTN_OK;
+}
+
+int sattn_debug_scores(const void *workspace, size_t ws_bytes, int B, int H, int N, int d, int mode, int32_t *out,
+                       sattn_stream_t stream) {
+  const int st = check_shape(B, H, N, d, mode);
+  if (st != SATTN_OK) return st;
+  if (is_nvfp4(mode)) return SATTN_ERR_UNSUPPORTED;
+  if (out == nullptr || (reinterpret_cast<uintptr_t>(out) & 15u)) return SATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
+  const sattn_ws_layout_t L = make_layout(B, H, N, d, mode);
+  if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
+  const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+  const int BH = B * H;
+  CUtensorMap tq, tk;
+  const CUtensorMapSwizzle sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map_u8(&tq, ws + L.q8, d, N, BH, d, static_cast<uint64_t>(N) * d, d, kTile, sw) ||
+      !make_map_u8(&tk, ws + L.k8, d, N, BH, d, static_cast<uint64_t>(N) * d, d, kTile, sw))
+    return SATTN_ERR_CUDA;
+  const int np = L.nblk * kTile;
+  const dim3 grid(L.nblk, L.nblk, BH);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 128)
+    debug_scores_kernel<128><<<grid, kDebugThreads, DebugScoresSmem<128>::kAlloc, cs>>>(tq, tk, out, np);
+  else
+    debug_scores_kernel<64><<<grid, kDebugThreads, DebugScoresSmem<64>::kAlloc, cs>>>(tq, tk, out, np);
+  g_launches += 1;
+  return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }
 
 int sattn_debug_withhold_statistics(int on) {

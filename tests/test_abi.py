@@ -152,6 +152,20 @@ def test_per_token_q_layout(L):
     assert L.sattn_workspace_bytes(2, 3, 1000, 128, NVFP4 | 0x400) == 0
 
 
+def test_scores_accessor_validates_before_any_cuda_call(L):
+    ws = ctypes.c_void_p(1 << 21)
+    out = ctypes.c_void_p(1 << 22)
+    f = L.sattn_debug_scores
+    f.argtypes = [ctypes.c_void_p, ctypes.c_size_t] + [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p]
+    assert f(ws, 1 << 30, 1, 2, 256, 64, NVFP4, out, None) == UNSUPPORTED
+    assert f(ws, 1 << 30, 1, 2, 256, 64, 2, out, None) == UNSUPPORTED           # MXFP4
+    assert f(ws, 1 << 30, 1, 2, 256, 64, BF16, None, None) == INVALID
+    assert f(ws, 1 << 30, 1, 2, 256, 64, BF16, ctypes.c_void_p((1 << 22) + 4), None) == INVALID
+    assert f(ws, 16, 1, 2, 256, 64, BF16, out, None) == WORKSPACE
+    assert f(None, 1 << 30, 1, 2, 256, 64, BF16, out, None) == WORKSPACE
+    assert f(ws, 1 << 30, 1, 2, 256, 96, BF16, out, None) == UNSUPPORTED
+
+
 def test_block_sparse_entry_points_validate_before_any_cuda_call(L):
     p = ctypes.c_void_p(1 << 20)
     o = ctypes.c_void_p(1 << 40)
