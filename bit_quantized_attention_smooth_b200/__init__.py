@@ -243,11 +243,13 @@ def fwd_host(q, k, v, causal=False, sm_scale=None, mode="i8f8", out=None, stream
 
 
 def debug_scores(workspace, shape, mode="i8f8", dtype=torch.bfloat16, stream=None, q_per_token=False):
-    """Test accessor: the INT8 scores q8 . k8^T of a quantised workspace,
-    int32 [B, H, Np, Np] (Np = N rounded up to 128), computed on the tensor cores."""
+    """Test accessor: the scores Q K^T of a quantised workspace computed on the
+    tensor cores, [B, H, Np, Np] (Np = N rounded up to 128): int32 q8 . k8^T
+    (I8QK_F8PV) or float32 products of the dequantised FP4 operands."""
     B, H, N, d = shape
     np_ = (N + 127) // 128 * 128
-    out = torch.empty((B, H, np_, np_), dtype=torch.int32, device=workspace.device)
+    out = torch.empty((B, H, np_, np_), dtype=torch.int32 if mode == "i8f8" else torch.float32,
+                      device=workspace.device)
     _check(lib().sattn_debug_scores(workspace.data_ptr(), workspace.numel(), B, H, N, d,
                                     mode_code(mode, dtype, q_per_token), out.data_ptr(), _stream(stream)),
            "sattn_debug_scores")

@@ -644,29 +644,57 @@ int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile) {
   return SATTN_OK;
 }
 
-int sattn_debug_scores(const void *workspace, size_t ws_bytes, int B, int H, int N, int d, int mode, int32_t *out,
+int sattn_debug_scores(const void *workspace, size_t ws_bytes, int B, int H, int N, int d, int mode, void *out,
                        sattn_stream_t stream) {
   const int st = check_shape(B, H, N, d, mode);
   if (st != SATTN_OK) return st;
-  if (is_nvfp4(mode)) return SATTN_ERR_UNSUPPORTED;
   if (out == nullptr || (reinterpret_cast<uintptr_t>(out) & 15u)) return SATTN_ERR_INVALID_ARG;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SATTN_ERR_WORKSPACE;
   const sattn_ws_layout_t L = make_layout(B, H, N, d, mode);
   if (ws_bytes < L.total) return SATTN_ERR_WORKSPACE;
   const uint8_t *ws = static_cast<const uint8_t *>(workspace);
   const int BH = B * H;
+  const int np = L.nblk * kTile;
+  const dim3 grid(L.nblk, L.nblk, BH);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (is_nvfp4(mode)) {                           // NVFP4 and MXFP4: float32 products of the dequantised codes
+    CUtensorMap tq, tk;
+    const CUtensorMapSwizzle swqk = d == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    const uint64_t rowb = d / 2;
+    if (!make_map_u8(&tq, ws + L.q8, rowb, N, BH, rowb, static_cast<uint64_t>(N) * rowb, rowb, kTile, swqk) ||
+        !make_map_u8(&tk, ws + L.k8, rowb, N, BH, rowb, static_cast<uint64_t>(N) * rowb, rowb, kTile, swqk))
+      return SATTN_ERR_CUDA;
+    float *o = static_cast<float *>(out);
+    const uint8_t *sfq = ws + L.sq, *sfk = ws + L.sk;
+    const bool mx = is_mxfp4(mode);
+    if (d == 128) {
+      if (mx)
+        debug_scores_fp4_kernel<128, true><<<grid, kDebugThreads, DebugScoresF4Smem<128>::kAlloc, cs>>>(
+            tq, tk, sfq, sfk, L.nblk, o, np);
+      else
+        debug_scores_fp4_kernel<128, false><<<grid, kDebugThreads, DebugScoresF4Smem<128>::kAlloc, cs>>>(
+            tq, tk, sfq, sfk, L.nblk, o, np);
+    } else {
+      if (mx)
+        debug_scores_fp4_kernel<64, true><<<grid, kDebugThreads, DebugScoresF4Smem<64>::kAlloc, cs>>>(
+            tq, tk, sfq, sfk, L.nblk, o, np);
+      else
+        debug_scores_fp4_kernel<64, false><<<grid, kDebugThreads, DebugScoresF4Smem<64>::kAlloc, cs>>>(
+            tq, tk, sfq, sfk, L.nblk, o, np);
+    }
+    g_launches += 1;
+    return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
+  }
   CUtensorMap tq, tk;
   const CUtensorMapSwizzle sw = d == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!make_map_u8(&tq, ws + L.q8, d, N, BH, d, static_cast<uint64_t>(N) * d, d, kTile, sw) ||
       !make_map_u8(&tk, ws + L.k8, d, N, BH, d, static_cast<uint64_t>(N) * d, d, kTile, sw))
     return SATTN_ERR_CUDA;
-  const int np = L.nblk * kTile;
-  const dim3 grid(L.nblk, L.nblk, BH);
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int32_t *o = static_cast<int32_t *>(out);
   if (d == 128)
-    debug_scores_kernel<128><<<grid, kDebugThreads, DebugScoresSmem<128>::kAlloc, cs>>>(tq, tk, out, np);
+    debug_scores_kernel<128><<<grid, kDebugThreads, DebugScoresSmem<128>::kAlloc, cs>>>(tq, tk, o, np);
   else
-    debug_scores_kernel<64><<<grid, kDebugThreads, DebugScoresSmem<64>::kAlloc, cs>>>(tq, tk, out, np);
+    debug_scores_kernel<64><<<grid, kDebugThreads, DebugScoresSmem<64>::kAlloc, cs>>>(tq, tk, o, np);
   g_launches += 1;
   return cudaGetLastError() == cudaSuccess ? SATTN_OK : SATTN_ERR_CUDA;
 }

@@ -255,18 +255,22 @@ int sattn_debug_set_wait_limit(long long cycles, int withhold_k_tile);
  * (it writes one device variable).  Returns SATTN_OK or SATTN_ERR_CUDA. */
 int sattn_debug_withhold_statistics(int on);
 
-/* Test accessor; not for production use.  Writes the integer scores of the
- * INT8 tensor-core product of the I8QK_F8PV mode (TurboDiffusion explainer,
- * section 1: QK^T in INT8), S_int[b, h, i, j] = sum_c q8[b, h, i, c] *
- * k8[b, h, j, c], of a workspace filled by sattn_quantize with the same
- * (B, H, N, d, mode): one 128 x 128 tile per CTA, loaded and multiplied with
- * the attention kernel's tensor maps, descriptors and tcgen05.mma kind::i8.
- * out: device memory, int32 [B*H, Np, Np], Np = ceil(N/128) * 128, 16-byte
- * aligned, owned by the caller; rows and columns at and past N hold products
- * of zero codes (0).  Asynchronous on `stream`, one launch.  NVFP4 / MXFP4:
- * SATTN_ERR_UNSUPPORTED; other errors as sattn_fwd_quantized. */
+/* Test accessor; not for production use.  Writes the scores S = Q K^T of
+ * the quantized operands of a workspace filled by sattn_quantize with the
+ * same (B, H, N, d, mode), computed on the tensor cores the way the attention
+ * kernels do (their tensor maps, descriptors and MMA kinds), one 128 x 128
+ * tile per CTA:
+ *   I8QK_F8PV: int32 S_int[b, h, i, j] = sum_c q8[b, h, i, c] k8[b, h, j, c]
+ *              (TurboDiffusion explainer, section 1: QK^T in INT8), exact;
+ *   NVFP4 / MXFP4: float32 sum_c Q^[i, c] K'^[j, c] of the dequantized E2M1
+ *              codes with their block scales applied by the block-scaled MMA
+ *              (tag page, SageAttention3 summary, FP4 bullet [15]).
+ * out: device memory [B*H, Np, Np], Np = ceil(N/128) * 128, of int32 or
+ * float32 as above, 16-byte aligned, owned by the caller; rows and columns at
+ * and past N hold products of zero codes (0).  Asynchronous on `stream`, one
+ * launch.  Errors as sattn_fwd_quantized. */
 int sattn_debug_scores(const void *workspace, size_t ws_bytes, int B, int H, int N, int d, int mode,
-                       int32_t *out, sattn_stream_t stream);
+                       void *out, sattn_stream_t stream);
 
 /* Number of CUDA kernels this library has launched, in this process, since it
  * was loaded or since the last call with reset != 0 (which returns the count

@@ -157,8 +157,8 @@ def test_scores_accessor_validates_before_any_cuda_call(L):
     out = ctypes.c_void_p(1 << 22)
     f = L.sattn_debug_scores
     f.argtypes = [ctypes.c_void_p, ctypes.c_size_t] + [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p]
-    assert f(ws, 1 << 30, 1, 2, 256, 64, NVFP4, out, None) == UNSUPPORTED
-    assert f(ws, 1 << 30, 1, 2, 256, 64, 2, out, None) == UNSUPPORTED           # MXFP4
+    assert f(ws, 16, 1, 2, 256, 64, NVFP4, out, None) == WORKSPACE
+    assert f(ws, 1 << 30, 1, 2, 256, 64, 2 | QTOK, out, None) == UNSUPPORTED    # MXFP4 with per-token Q
     assert f(ws, 1 << 30, 1, 2, 256, 64, BF16, None, None) == INVALID
     assert f(ws, 1 << 30, 1, 2, 256, 64, BF16, ctypes.c_void_p((1 << 22) + 4), None) == INVALID
     assert f(ws, 16, 1, 2, 256, 64, BF16, out, None) == WORKSPACE

@@ -1,4 +1,4 @@
-"""The INT8 tensor-core product of the I8QK_F8PV mode, bit for bit.
+"""The tensor-core products S = Q K^T of the quantised operands.
 
 S_int = q8 . k8^T is the one exact integer step of the attention (TurboDiffusion
 explainer, section 1: QK^T in INT8).  sattn_debug_scores runs it the way the
@@ -6,7 +6,8 @@ attention kernel does (same TMA tensor maps and swizzle, same shared-memory and
 instruction descriptors, tcgen05.mma kind::i8 into tensor memory) and exports
 the int32 accumulator.  It must equal the exact integer product of the oracle's
 own INT8 codes of the same inputs, element by element; rows and columns past N
-(zero-filled tiles) must be 0.
+(zero-filled tiles) must be 0.  The FP4 modes' block-scaled product is checked
+against the float64 product of the oracle's dequantised operands.
 """
 
 import numpy as np
@@ -54,9 +55,33 @@ def test_int8_scores_bit_exact(w, q_per_token):
             assert np.array_equal(got[b, h, :N, :N].astype(np.int64), want), (b, h)
 
 
-def test_scores_accessor_rejects_fp4_modes():
-    w = W.custom(1, 1, 128, 64, seed=75)
+@pytest.mark.parametrize("w,mode", [
+    (W.custom(1, 2, 300, 128, seed=76, q_outlier_frac=1e-3), "nvfp4"),
+    (W.custom(2, 1, 129, 64, "fp16", seed=77), "nvfp4"),
+    (W.custom(1, 2, 300, 128, seed=78, q_outlier_frac=1e-3), "mxfp4"),
+    (W.custom(1, 1, 200, 64, seed=79), "mxfp4"),
+], ids=lambda x: getattr(x, "name", str(x)))
+def test_fp4_scores_are_the_dequantised_product(w, mode):
+    """The block-scaled MMA applies the scale factors where the oracle puts
+    them: S equals the float64 product of the oracle's dequantised operands up
+    to float32 accumulation (1e-5 of the sum of |terms|).  For MXFP4 this pins
+    the E8M0 codes stored at both 16-value positions of each 32-value block."""
     q, k, v = W.make_inputs(w, "cuda")
-    ws = sattn.quantize(q, k, v, mode="nvfp4")
-    with pytest.raises(sattn.SattnError):
-        sattn.debug_scores(ws, q.shape, mode="nvfp4", dtype=q.dtype)
+    ws = sattn.quantize(q, k, v, mode=mode)
+    s = sattn.debug_scores(ws, q.shape, mode=mode, dtype=q.dtype)
+    torch.cuda.synchronize()
+    got = s.cpu().numpy().astype(np.float64)
+    N, d = w.N, w.d
+    assert not np.any(got[:, :, N:, :]) and not np.any(got[:, :, :, N:])
+    qf, kf, vf = (t.float().cpu().numpy() for t in (q, k, v))
+    head = Qz.quantize_head_nvfp4 if mode == "nvfp4" else Qz.quantize_head_mxfp4
+    blk = 16 if mode == "nvfp4" else 32
+    for b in range(w.B):
+        for h in range(w.H):
+            z = head(qf[b, h], kf[b, h], vf[b, h])
+            qv = Qz.nvfp4_dequant_rows(z["q"], z["q_sc"], block=blk)[:, :d]
+            kv = Qz.nvfp4_dequant_rows(z["k"], z["k_sc"], block=blk)[:, :d]
+            want = qv @ kv.T
+            bound = np.abs(qv) @ np.abs(kv).T
+            err = np.abs(got[b, h, :N, :N] - want)
+            assert np.all(err <= 1e-5 * bound), (b, h, float((err / np.maximum(bound, 1e-300)).max()))
